@@ -1,0 +1,148 @@
+"""FP64 CPU oracle for the Whisper-style attention pass.
+
+TEST INFRASTRUCTURE. Only the tests, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+module. The CUDA library never calls it and shares no code with it.
+
+What it computes is the plain definition, step by step, in float64 with no
+blocking, fusion or reordering beyond what the definition states. NumPy's
+matmul serves as the library primitive for the dot products.
+
+* Packed QKV projection -- the edda PR ("Add Edda ASR with DFlash2 speculative
+  decoding", PR description and the commit note on the encoder) replaces three
+  projections by one packed one. With the packed weight W (q rows, then k rows,
+  then v rows): qkv[r, j] = sum_c x[r, c] * W[j, c] + bias[j], where bias is b_q
+  on the q third, 0 on the k third (Whisper's key projection has no bias) and
+  b_v on the v third.
+* Scaled-dot-product attention with a per-row allowed set A_i. The PR's flash
+  path gives the same transcripts as the path that materialises the scores, so
+  the oracle materialises them: s_ij = scale * <q_i, k_j>, m_i = max over A_i,
+  p_ij = exp(s_ij - m_i) on A_i and 0 elsewhere, l_i = sum_j p_ij,
+  o_i = sum_j p_ij v_j / l_i. A row whose allowed set is empty yields 0 (the
+  pages are silent on that case; zero is the reading taken).
+* Allowed sets: FULL = every key (the Whisper encoder is fully bidirectional:
+  BuzzASR "danish" discussion #1, the reply on the padded region); CHUNK(len) =
+  keys in the same len-frame chunk of the same sequence (higgs-audio-v3-stt model
+  card, "Architecture note (chunked encoder)": each chunk is encoded on its own
+  with within-chunk attention); SLOTMASK = the explicit per-row bitmask of a
+  token tree over a position-indexed cache (edda PR description: each beam's
+  mask row admits only its ancestors; block verification over KV slots indexed
+  by position).
+
+Inputs arrive as fp16 arrays and are widened to float64 exactly. Nothing is
+rounded in between; the output stays float64.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+HEAD_DIM = 64
+
+
+def _f64(a: np.ndarray) -> np.ndarray:
+    return np.asarray(a).astype(np.float64)
+
+
+def packed_bias(b_q: np.ndarray, b_v: np.ndarray) -> np.ndarray:
+    """The 3d-long bias of the packed projection: [b_q | 0 | b_v]."""
+    b_q = _f64(b_q)
+    return np.concatenate([b_q, np.zeros_like(b_q), _f64(b_v)])
+
+
+def qkv_projection(x: np.ndarray, w_qkv: np.ndarray, b_q: np.ndarray, b_v: np.ndarray) -> np.ndarray:
+    """qkv = x . W^T + [b_q | 0 | b_v] in float64.  x [rows, d], W [3d, d] -> [rows, 3d]."""
+    return _f64(x) @ _f64(w_qkv).T + packed_bias(b_q, b_v)
+
+
+# ----------------------------------------------------------------------------
+# allowed sets
+# ----------------------------------------------------------------------------
+
+def allowed_full(t_q: int, t_kv: int) -> np.ndarray:
+    return np.ones((t_q, t_kv), dtype=bool)
+
+
+def allowed_chunk(t: int, chunk_len: int) -> np.ndarray:
+    """allowed(i, j) <=> floor(i / len) == floor(j / len), frames counted from the
+    start of the sequence; the last chunk may be short."""
+    if chunk_len <= 0:
+        raise ValueError("chunk_len must be positive")
+    c = np.arange(t) // chunk_len
+    return c[:, None] == c[None, :]
+
+
+def allowed_from_bits(bits: np.ndarray, t_kv: int) -> np.ndarray:
+    """allowed(i, j) <=> bit (j % 32) of word (j // 32) of row i is set."""
+    bits = np.asarray(bits, dtype=np.uint32)
+    j = np.arange(t_kv)
+    return ((bits[:, j // 32] >> (j % 32).astype(np.uint32)) & 1).astype(bool)
+
+
+# ----------------------------------------------------------------------------
+# attention
+# ----------------------------------------------------------------------------
+
+def attention_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, allowed: np.ndarray,
+                   scale: float, return_stats: bool = False):
+    """One head: q [t_q, dh], k/v [t_kv, dh] (float64), allowed [t_q, t_kv]."""
+    s = scale * (q @ k.T)
+    s_masked = np.where(allowed, s, -np.inf)
+    nonempty = allowed.any(axis=1)
+    m = np.where(nonempty, s_masked.max(axis=1), 0.0)
+    p = np.where(allowed, np.exp(s_masked - m[:, None]), 0.0)
+    l = p.sum(axis=1)
+    o = np.zeros((q.shape[0], v.shape[1]), dtype=np.float64)
+    o[nonempty] = (p[nonempty] @ v) / l[nonempty, None]
+    if return_stats:
+        return o, {"s": s, "m": m, "l": l, "p": p}
+    return o
+
+
+def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, n_heads: int, allowed: np.ndarray,
+              scale: float = 1.0 / np.sqrt(HEAD_DIM), head_dim: int = HEAD_DIM,
+              return_stats: bool = False):
+    """Multi-head attention for one sequence. q [t_q, H*dh], k/v [t_kv, H*dh];
+    head h uses columns [h*dh, (h+1)*dh) of each. Returns o [t_q, H*dh] float64."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    o = np.zeros((q.shape[0], n_heads * head_dim), dtype=np.float64)
+    stats = []
+    for h in range(n_heads):
+        cols = slice(h * head_dim, (h + 1) * head_dim)
+        res = attention_head(q[:, cols], k[:, cols], v[:, cols], allowed, scale, return_stats)
+        if return_stats:
+            o[:, cols], st = res
+            stats.append(st)
+        else:
+            o[:, cols] = res
+    if return_stats:
+        return o, stats
+    return o
+
+
+def encoder_attention(x: np.ndarray, w_qkv: np.ndarray, b_q: np.ndarray, b_v: np.ndarray,
+                      batch: int, t: int, n_heads: int, mask: str = "full", chunk_len: int = 0,
+                      scale: float = 1.0 / np.sqrt(HEAD_DIM), return_qkv: bool = False):
+    """Packed projection followed by self-attention of each of ``batch``
+    sequences of ``t`` frames. mask is "full" or "chunk"."""
+    d = x.shape[1]
+    qkv = qkv_projection(x, w_qkv, b_q, b_v)
+    allowed = allowed_full(t, t) if mask == "full" else allowed_chunk(t, chunk_len)
+    out = np.zeros((batch * t, d), dtype=np.float64)
+    for b in range(batch):
+        rows = slice(b * t, (b + 1) * t)
+        out[rows] = attention(qkv[rows, :d], qkv[rows, d:2 * d], qkv[rows, 2 * d:], n_heads, allowed, scale)
+    if return_qkv:
+        return out, qkv
+    return out
+
+
+def slotmask_attention(q, k_cache, v_cache, bits, n_heads, scale=1.0 / np.sqrt(HEAD_DIM)):
+    """Block verification over a position-indexed cache with an explicit
+    allowed-slot bitmask (one row of words per query row, shared by all heads)."""
+    return attention(q, k_cache, v_cache, n_heads, allowed_from_bits(bits, k_cache.shape[0]), scale)
+
+
+def cross_attention(q, k_enc, v_enc, n_heads, scale=1.0 / np.sqrt(HEAD_DIM)):
+    """Decoder queries attending to every encoder frame (t_q != t_kv allowed)."""
+    return attention(q, k_enc, v_enc, n_heads, allowed_full(q.shape[0], k_enc.shape[0]), scale)
+

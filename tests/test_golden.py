@@ -1,0 +1,25 @@
+"""The oracle against its stored regression fixture (written by
+tests/golden/make_golden.py from the oracle alone)."""
+import json
+import os
+
+import numpy as np
+
+import oracle
+from speech_encoder_attention_b200 import inputs
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def test_tiny_oracle_matches_fixture():
+    with open(os.path.join(HERE, "golden", "tiny_oracle.json")) as f:
+        doc = json.load(f)
+    spec = inputs.ENCODER_WORKLOADS["tiny"]
+    inp = inputs.make_encoder_inputs(spec)
+    out, qkv = oracle.encoder_attention(inp.x, inp.w_qkv, inp.b_q, inp.b_v, 1, 64, 2, return_qkv=True)
+    for r, c, val in doc["out"]:
+        assert abs(out[r, c] - val) <= 1e-12 * max(1.0, abs(val))
+    for r, c, val in doc["qkv"]:
+        assert abs(qkv[r, c] - val) <= 1e-12 * max(1.0, abs(val))
+    assert abs(np.linalg.norm(out) - doc["out_l2"]) <= 1e-10
+    assert abs(np.linalg.norm(qkv) - doc["qkv_l2"]) <= 1e-10

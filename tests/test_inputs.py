@@ -1,0 +1,85 @@
+"""The seeded generators: determinism, shapes, distributions and the token tree."""
+import numpy as np
+
+from speech_encoder_attention_b200 import inputs
+
+
+def test_encoder_inputs_are_deterministic_and_shaped():
+    spec = inputs.ENCODER_WORKLOADS["tiny"]
+    a = inputs.make_encoder_inputs(spec)
+    b = inputs.make_encoder_inputs(spec)
+    assert a.x.shape == (64, 128) and a.w_qkv.shape == (384, 128)
+    assert a.b_q.shape == (128,) and a.b_v.shape == (128,)
+    assert a.x.dtype == np.float16
+    for f in ("x", "w_qkv", "b_q", "b_v"):
+        np.testing.assert_array_equal(getattr(a, f), getattr(b, f))
+
+
+def test_batch_override_keeps_leading_windows():
+    spec = inputs.ENCODER_WORKLOADS["windows8"]
+    small = inputs.make_encoder_inputs(spec, batch=2)
+    assert small.x.shape == (3000, 1280)
+    full = inputs.make_encoder_inputs(spec)
+    np.testing.assert_array_equal(full.x[:3000], small.x)
+    np.testing.assert_array_equal(full.w_qkv, small.w_qkv)
+
+
+def test_window_offsets_differ_per_window():
+    full = inputs.make_encoder_inputs(inputs.ENCODER_WORKLOADS["windows8"])
+    means = full.x.astype(np.float64).reshape(8, 1500, 1280).mean(axis=(1, 2))
+    assert np.all(np.abs(means) < 0.55)
+    assert np.ptp(means) > 0.1
+
+
+def test_distributions():
+    full = inputs.make_encoder_inputs(inputs.ENCODER_WORKLOADS["window"])
+    assert abs(full.x.astype(np.float64).std() - 1.0) < 0.01
+    assert abs(full.w_qkv.astype(np.float64).std() - 0.02) < 0.001
+    assert abs(full.b_q.astype(np.float64).std() - 0.01) < 0.002
+
+
+def test_chunk_workload_is_eleven_full_chunks_and_a_short_one():
+    spec = inputs.ENCODER_WORKLOADS["chunks"]
+    assert spec.t == 11 * 200 + 125 and spec.chunk_len == 200
+
+
+def test_token_tree_shape_and_counts():
+    spec = inputs.VERIFY_WORKLOADS["verify"]
+    inp = inputs.make_verify_inputs(spec)
+    assert spec.t_q == 80 and spec.slots == 448
+    assert inp.bits.shape == (80, 14) and inp.bits.dtype == np.uint32
+    allowed = inputs.unpack_bits(inp.bits, 448)
+    counts = allowed.sum(axis=1)
+    # prompt (8) + one slot per beam step (72) + position in the block (1..16)
+    np.testing.assert_array_equal(counts, np.tile(np.arange(81, 97), 5))
+    assert counts.sum() == 7080
+    # every row admits itself and the whole prompt, and nothing after itself
+    for r, s in enumerate(inp.query_slot):
+        assert allowed[r, s]
+        assert allowed[r, :8].all()
+        assert not allowed[r, s + 1:].any()
+    # beams do not see each other's blocks
+    for b in range(5):
+        rows = slice(16 * b, 16 * b + 16)
+        for b2 in range(5):
+            if b2 != b:
+                assert not allowed[rows, 368 + 16 * b2: 368 + 16 * b2 + 16].any()
+
+
+def test_token_tree_parents_are_earlier_slots():
+    spec = inputs.VERIFY_WORKLOADS["verify"]
+    inp = inputs.make_verify_inputs(spec)
+    p = inp.parent
+    assert p[0] == -1
+    assert np.all(p[1:] < np.arange(1, len(p)))
+    assert np.all(p[1:] >= 0)
+
+
+def test_pack_unpack_roundtrip():
+    rng = np.random.default_rng(0)
+    a = rng.random((7, 70)) < 0.5
+    np.testing.assert_array_equal(inputs.unpack_bits(inputs.pack_bits(a), 70), a)
+    bits = inputs.pack_bits(a)
+    assert bits.shape == (7, 3)
+    # bits past the last slot stay clear
+    assert np.all(bits[:, 2] >> np.uint32(6) == 0)
