@@ -1,0 +1,163 @@
+/*
+ * attn.h -- C ABI of libattn.so: the Whisper-style attention pass on B200 (sm_100a).
+ *
+ * The pass has two stages, both hand-written CUDA kernels for sm_100a:
+ *   1. a packed QKV projection (one GEMM instead of three), and
+ *   2. fused multi-head flash attention with fp16 K/V, an fp32 online softmax
+ *      and no score matrix in memory, under one of three masks.
+ * Sources (page titles and sections):
+ *   - "Add Edda ASR with DFlash2 speculative decoding" (audio.cpp PR #1223), PR
+ *     description: the encoder packs QKV and runs flash attention over F16 K/V
+ *     instead of materialising F32 scores for all 1500 frames; block verification
+ *     of an anchor plus up to 15 drafted tokens against KV slots indexed by
+ *     position; a token-tree KV cache whose mask rows admit only ancestors; the
+ *     drafter's flash cross-attention.
+ *   - "higgs-audio-v3-stt GGUF" model card, "Architecture note (chunked encoder)":
+ *     4 s chunks encoded independently with within-chunk attention.
+ *   - BuzzASR "danish" discussion #1: the Whisper encoder is fully bidirectional.
+ *
+ * Conventions for every entry point
+ *   - All tensors are IEEE fp16 (binary16) in device memory unless stated.
+ *   - A matrix is passed as attn_mat {ptr, row_stride}: element (r, c) lives at
+ *     ptr[r * row_stride + c]; row_stride counts elements. Sequence b of a batch
+ *     of sequences of length t occupies rows [b*t, (b+1)*t).
+ *   - Head h of a [rows, n_heads*64] matrix uses columns [64h, 64h+64).
+ *   - The caller owns every buffer, including the workspace. The library
+ *     allocates no device memory, keeps no per-call state and never
+ *     synchronises: all work is enqueued on `stream` in order and the call
+ *     returns immediately.
+ *   - Arguments are validated on the host before anything is launched. An
+ *     invalid argument returns ATTN_ERR_INVALID and launches nothing; there is
+ *     no fallback path. A launch failure returns ATTN_ERR_CUDA.
+ *   - Device pointers must be 16-byte aligned and row strides multiples of 8
+ *     elements (the tensor-memory-accelerator copies need 16-byte strides).
+ *   - No C++ exception crosses this interface.
+ */
+#ifndef SEA_ATTN_H
+#define SEA_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL means the legacy default stream. */
+typedef struct CUstream_st *attn_stream_t;
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID = 1,     /* bad argument; nothing was launched */
+  ATTN_ERR_UNSUPPORTED = 2, /* valid request this build does not serve (e.g. no sm_100 device) */
+  ATTN_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+  ATTN_ERR_TIMEOUT = 4      /* a kernel's bounded wait expired (see attn_debug_error_word) */
+} attn_status;
+
+typedef enum {
+  ATTN_MASK_FULL = 0,     /* every key: the bidirectional encoder window */
+  ATTN_MASK_CHUNK = 1,    /* keys in the query's chunk of chunk_len frames */
+  ATTN_MASK_SLOTMASK = 2  /* keys whose bit is set in the query row's bitmask */
+} attn_mask_kind;
+
+typedef struct {
+  int32_t kind;            /* attn_mask_kind */
+  int32_t chunk_len;       /* CHUNK: frames per chunk, > 0. Chunks start at frame 0
+                              of each sequence; the last one may be short. */
+  const uint32_t *bits;    /* SLOTMASK: device pointer, [t_q, words_per_row] uint32.
+                              Slot j of row i is allowed iff bit (j % 32) of word
+                              i*words_per_row + j/32 is set (LSB first). Shared by
+                              all heads and all sequences of the batch. 4-byte aligned. */
+  int32_t words_per_row;   /* SLOTMASK: >= ceil(t_kv / 32) */
+  int32_t reserved;        /* must be 0 */
+} attn_mask;
+
+typedef struct {
+  void *ptr;               /* device pointer (read-only for inputs) */
+  int64_t row_stride;      /* elements between consecutive rows */
+} attn_mat;
+
+/*
+ * attn_qkv_pack -- the packed QKV projection
+ *   qkv[r, j] = sum_c x[r, c] * W[j, c] + bias[j],  bias = [b_q | 0 | b_v]
+ * Source: the edda PR description ("packs QKV"): one projection with the packed
+ * weight W = [W_q; W_k; W_v] instead of three. As in Whisper, the key projection
+ * has no bias.
+ *   x        [rows, d_model]    fp16, row_stride >= d_model
+ *   w_qkv    [3*d_model, d_model] fp16, contiguous (q rows, k rows, v rows)
+ *   b_q, b_v [d_model] fp16, may be NULL (treated as zero)
+ *   qkv_out  [rows, 3*d_model]  fp16, row_stride >= 3*d_model; must not overlap x or W
+ * d_model must be a positive multiple of 64 and rows >= 1. Accumulates in fp32,
+ * adds the bias in fp32 and rounds once to fp16 (round to nearest even).
+ */
+attn_status attn_qkv_pack(attn_mat x, const void *w_qkv, const void *b_q, const void *b_v,
+                          int64_t rows, int32_t d_model, attn_mat qkv_out, attn_stream_t stream);
+
+/*
+ * attn_forward -- multi-head flash attention with a mask
+ *   o_i = sum_{j in A_i} softmax_j(scale * <q_i, k_j>) v_j     per head
+ * A_i by mask.kind: FULL -> all t_kv keys; CHUNK -> keys of the same chunk
+ * (requires t_q == t_kv); SLOTMASK -> keys whose bit is set in row i. A row
+ * with an empty A_i yields zeros.
+ *   q   [batch*t_q,  n_heads*64] fp16   (row_stride >= n_heads*64)
+ *   k,v [batch*t_kv, n_heads*64] fp16
+ *   out [batch*t_q,  n_heads*64] fp16, must not overlap q, k or v
+ * q, k and v may be three views of one packed projection buffer (row_stride
+ * 3*d_model, pointers at column offsets 0, d_model and 2*d_model).
+ * head_dim must be 64. Scores, the running max and sum and the output
+ * accumulate in fp32; the softmax weights are rounded to fp16 for the value
+ * product; the output is rounded once to fp16.
+ * workspace: device scratch of at least attn_workspace_size(...) bytes, 16-byte
+ * aligned, used to split long key ranges of short query blocks over more SMs.
+ * Passing workspace == NULL with workspace_bytes == 0 disables the split (the
+ * result is the same, only the schedule differs); a non-NULL workspace smaller
+ * than required returns ATTN_ERR_INVALID.
+ */
+attn_status attn_forward(attn_mat q, attn_mat k, attn_mat v, int32_t batch, int32_t t_q,
+                         int32_t t_kv, int32_t n_heads, int32_t head_dim, attn_mask mask,
+                         float scale, attn_mat out, void *workspace, size_t workspace_bytes,
+                         attn_stream_t stream);
+
+/*
+ * attn_cross -- decoder queries attending to every encoder frame
+ * Source: the edda PR description (the drafter's flash cross-attention); the
+ * decoder attends over the whole encoded sequence (higgs model card note).
+ * Same as attn_forward with a FULL mask and t_kv = t_enc (t_q != t_enc allowed).
+ *   q [batch*t_q, n_heads*64], k_enc, v_enc [batch*t_enc, n_heads*64], out like q.
+ */
+attn_status attn_cross(attn_mat q, attn_mat k_enc, attn_mat v_enc, int32_t batch, int32_t t_q,
+                       int32_t t_enc, int32_t n_heads, int32_t head_dim, float scale,
+                       attn_mat out, void *workspace, size_t workspace_bytes,
+                       attn_stream_t stream);
+
+/*
+ * attn_workspace_size -- bytes of workspace attn_forward / attn_cross use for
+ * these sizes on the current device (0 when no split is planned).
+ */
+size_t attn_workspace_size(int32_t batch, int32_t t_q, int32_t t_kv, int32_t n_heads,
+                           int32_t head_dim, int32_t mask_kind);
+
+/* Static, human-readable name of a status code. */
+const char *attn_status_string(attn_status status);
+
+/*
+ * attn_debug_error_word -- synchronises `stream`, then reads and clears the
+ * device error word that kernels set when a bounded wait expires. Writes the
+ * raw word to *word_out when word_out is not NULL. Returns ATTN_ERR_TIMEOUT if
+ * it was set, ATTN_OK otherwise.
+ */
+attn_status attn_debug_error_word(attn_stream_t stream, uint32_t *word_out);
+
+/*
+ * attn_debug_timeout_probe -- launches one tiny kernel that waits on a barrier
+ * nothing will ever complete, with a limit of limit_ns nanoseconds (1e3..1e9).
+ * The kernel gives up, records the timeout in the error word and returns, so
+ * the context stays usable. A test of the bounded-wait path, with no fault.
+ */
+attn_status attn_debug_timeout_probe(int64_t limit_ns, attn_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SEA_ATTN_H */

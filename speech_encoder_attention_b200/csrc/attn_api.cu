@@ -1,0 +1,388 @@
+// attn_api.cu -- the C ABI of libattn.so (declared in include/attn.h).
+//
+// Host side of the library: argument validation, the launch plan (query-tile
+// schedule, key/value split), TMA tensor-map encoding and kernel launches.
+// Everything is enqueued on the caller's stream; nothing here allocates device
+// memory or synchronises (except the two debug entry points, which say so).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "attn.h"
+#include "flash_attn.cuh"
+#include "qkv_gemm.cuh"
+#include "sm100_ptx.cuh"
+
+namespace {
+
+// Device-side error word: kernels OR kErrTimeout into it when a bounded wait
+// gives up. One copy per device.
+__device__ uint32_t g_error_word = 0;
+
+// Waits on a barrier nothing will complete, so the bounded-wait path can be
+// tested without hanging or faulting the GPU.
+__global__ void timeout_probe_kernel(uint32_t* err, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ uint32_t abort_flag;
+  if (threadIdx.x == 0) {
+    sea::mbar_init(sea::smem_u32(&bar), 1);
+    abort_flag = 0u;
+    sea::fence_barrier_init();
+  }
+  __syncthreads();
+  const sea::WaitCtl wc{&abort_flag, err, limit_ns};
+  sea::mbar_wait(sea::smem_u32(&bar), 0, wc);
+}
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ok = false;       // sm_100 device, attributes set
+  int num_sms = 0;
+  uint32_t* err = nullptr;  // address of g_error_word on this device
+};
+
+std::mutex g_mutex;
+DeviceInfo g_dev[kMaxDevices];
+bool g_dev_init[kMaxDevices] = {};
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode;
+}
+
+// Per-device set-up: checks for an sm_100 part, records the SM count and the
+// error-word address, and raises the dynamic shared-memory limits once.
+attn_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceInfo& d = g_dev[dev];
+  if (!g_dev_init[dev]) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    g_dev_init[dev] = true;
+    if (major != 10 || minor != 0) return ATTN_ERR_UNSUPPORTED;
+    void* err = nullptr;
+    if (cudaGetSymbolAddress(&err, g_error_word) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (cudaFuncSetAttribute(sea::gemm::qkv_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             sea::gemm::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(sea::fa::flash_attn_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             sea::fa::Cfg<1>::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(sea::fa::flash_attn_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             sea::fa::Cfg<2>::SMEM_BYTES) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    d.num_sms = sms;
+    d.err = static_cast<uint32_t*>(err);
+    d.ok = true;
+  }
+  if (!d.ok) return ATTN_ERR_UNSUPPORTED;
+  *out = &d;
+  return ATTN_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Byte range [lo, hi) touched by a row-major fp16 matrix.
+struct Range {
+  uintptr_t lo, hi;
+};
+Range mat_range(const void* p, int64_t rows, int64_t cols, int64_t stride) {
+  const uintptr_t lo = reinterpret_cast<uintptr_t>(p);
+  return {lo, lo + static_cast<uintptr_t>(((rows - 1) * stride + cols) * 2)};
+}
+bool overlaps(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi; }
+
+bool encode_2d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t stride_bytes,
+               uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
+  auto enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {stride_bytes};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// (columns, frames, sequence) view of a [batch*t, >=cols] matrix: rows past a
+// sequence's end read as zeros instead of the next sequence's frames.
+bool encode_seq_3d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t t, uint64_t batch,
+                   uint64_t row_stride_elems) {
+  auto enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {cols, t, batch};
+  cuuint64_t strides[2] = {row_stride_elems * 2, row_stride_elems * 2 * t};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct FaPlan {
+  int nq;
+  int seg_len, tiles_per_seg, q_tiles;
+  int n_kv_max;
+  int kv_splits, kv_tiles_per_split;
+  size_t ws_bytes;
+};
+
+int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
+
+// Launch plan shared by attn_forward and attn_workspace_size.
+FaPlan plan_forward(int batch, int t_q, int t_kv, int n_heads, int mask_kind, int chunk_len, int num_sms) {
+  FaPlan pl{};
+  const bool chunked = mask_kind == sea::fa::kChunk && chunk_len < t_q;
+  if (chunked) {
+    // Segments of whole chunks: one chunk when it is at least a tile long,
+    // otherwise as many whole chunks as fit in 128 rows.
+    pl.seg_len = chunk_len >= sea::fa::BQ ? chunk_len : (sea::fa::BQ / chunk_len) * chunk_len;
+    pl.tiles_per_seg = ceil_div(pl.seg_len, sea::fa::BQ);
+    pl.q_tiles = ceil_div(t_q, pl.seg_len) * pl.tiles_per_seg;
+    pl.nq = (pl.tiles_per_seg % 2 == 0) ? 2 : 1;
+    pl.n_kv_max = ceil_div(pl.seg_len, sea::fa::BKV) + 1;
+  } else {
+    pl.seg_len = t_q;
+    pl.tiles_per_seg = ceil_div(t_q, sea::fa::BQ);
+    pl.q_tiles = pl.tiles_per_seg;
+    pl.nq = pl.q_tiles >= 2 ? 2 : 1;
+    pl.n_kv_max = ceil_div(t_kv, sea::fa::BKV);
+  }
+  pl.kv_splits = 1;
+  pl.kv_tiles_per_split = pl.n_kv_max;
+  const int64_t base_ctas = static_cast<int64_t>(batch) * n_heads * ceil_div(pl.q_tiles, pl.nq);
+  // CHUNK tiles already fill the GPU; the split serves short query blocks.
+  if (mask_kind != sea::fa::kChunk && base_ctas * 2 <= num_sms && pl.n_kv_max >= 2) {
+    int splits = static_cast<int>(std::min<int64_t>(pl.n_kv_max, std::max<int64_t>(1, num_sms / base_ctas)));
+    const int per = ceil_div(pl.n_kv_max, splits);
+    splits = ceil_div(pl.n_kv_max, per);
+    if (splits > 1) {
+      pl.kv_splits = splits;
+      pl.kv_tiles_per_split = per;
+      const size_t rows = static_cast<size_t>(splits) * batch * n_heads * t_q;
+      pl.ws_bytes = rows * sea::fa::DH * sizeof(float) + rows * 2 * sizeof(float);
+    }
+  }
+  return pl;
+}
+
+bool valid_mat(const attn_mat& m, int64_t cols) {
+  return m.ptr != nullptr && aligned16(m.ptr) && m.row_stride >= cols && (m.row_stride % 8) == 0;
+}
+
+attn_status launch_attention(attn_mat q, attn_mat k, attn_mat v, int32_t batch, int32_t t_q, int32_t t_kv,
+                             int32_t n_heads, int32_t head_dim, attn_mask mask, float scale, attn_mat out,
+                             void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  // ---- validation (host only, before any CUDA call) ----
+  if (batch <= 0 || t_q <= 0 || t_kv <= 0 || n_heads <= 0) return ATTN_ERR_INVALID;
+  if (head_dim != sea::fa::DH) return ATTN_ERR_INVALID;
+  if (batch > 65535 || n_heads > 65535) return ATTN_ERR_INVALID;
+  if (static_cast<int64_t>(batch) * t_q > INT32_MAX || static_cast<int64_t>(batch) * t_kv > INT32_MAX)
+    return ATTN_ERR_INVALID;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID;
+  const int64_t cols = static_cast<int64_t>(n_heads) * head_dim;
+  if (!valid_mat(q, cols) || !valid_mat(k, cols) || !valid_mat(v, cols) || !valid_mat(out, cols))
+    return ATTN_ERR_INVALID;
+  if (mask.reserved != 0) return ATTN_ERR_INVALID;
+  if (mask.kind == ATTN_MASK_CHUNK) {
+    if (mask.chunk_len <= 0 || t_q != t_kv) return ATTN_ERR_INVALID;
+  } else if (mask.kind == ATTN_MASK_SLOTMASK) {
+    if (mask.bits == nullptr || (reinterpret_cast<uintptr_t>(mask.bits) & 3u) != 0) return ATTN_ERR_INVALID;
+    if (t_kv > sea::fa::MAX_FLAG_WORDS * 32 * sea::fa::BKV) return ATTN_ERR_INVALID;
+    if (mask.words_per_row < (t_kv + 31) / 32) return ATTN_ERR_INVALID;
+  } else if (mask.kind != ATTN_MASK_FULL) {
+    return ATTN_ERR_INVALID;
+  }
+  const Range ro = mat_range(out.ptr, static_cast<int64_t>(batch) * t_q, cols, out.row_stride);
+  if (overlaps(ro, mat_range(q.ptr, static_cast<int64_t>(batch) * t_q, cols, q.row_stride)) ||
+      overlaps(ro, mat_range(k.ptr, static_cast<int64_t>(batch) * t_kv, cols, k.row_stride)) ||
+      overlaps(ro, mat_range(v.ptr, static_cast<int64_t>(batch) * t_kv, cols, v.row_stride)))
+    return ATTN_ERR_INVALID;
+  if (workspace != nullptr && !aligned16(workspace)) return ATTN_ERR_INVALID;
+  if (workspace == nullptr && workspace_bytes != 0) return ATTN_ERR_INVALID;
+
+  DeviceInfo* dev = nullptr;
+  if (attn_status st = device_info(&dev); st != ATTN_OK) return st;
+
+  FaPlan pl = plan_forward(batch, t_q, t_kv, n_heads, mask.kind, mask.chunk_len, dev->num_sms);
+  if (pl.kv_splits > 1) {
+    if (workspace == nullptr) {
+      pl.kv_splits = 1;  // caller opted out of the split: same result, one CTA per key range
+      pl.kv_tiles_per_split = pl.n_kv_max;
+      pl.ws_bytes = 0;
+    } else if (workspace_bytes < pl.ws_bytes) {
+      return ATTN_ERR_INVALID;
+    }
+  }
+
+  CUtensorMap tq, tk, tv;
+  if (!encode_seq_3d(&tq, q.ptr, cols, t_q, batch, q.row_stride) ||
+      !encode_seq_3d(&tk, k.ptr, cols, t_kv, batch, k.row_stride) ||
+      !encode_seq_3d(&tv, v.ptr, cols, t_kv, batch, v.row_stride))
+    return ATTN_ERR_CUDA;
+
+  sea::fa::Params p{};
+  p.batch = batch;
+  p.t_q = t_q;
+  p.t_kv = t_kv;
+  p.n_heads = n_heads;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.mask_kind = mask.kind;
+  p.chunk_len = (mask.kind == ATTN_MASK_CHUNK && mask.chunk_len < t_q) ? mask.chunk_len : t_q;
+  if (mask.kind == ATTN_MASK_CHUNK && mask.chunk_len >= t_q) p.mask_kind = sea::fa::kFull;
+  p.bits = mask.kind == ATTN_MASK_SLOTMASK ? mask.bits : nullptr;
+  p.words_per_row = mask.kind == ATTN_MASK_SLOTMASK ? mask.words_per_row : 0;
+  p.seg_len = pl.seg_len;
+  p.tiles_per_seg = pl.tiles_per_seg;
+  p.q_tiles = pl.q_tiles;
+  p.kv_splits = pl.kv_splits;
+  p.kv_tiles_per_split = pl.kv_tiles_per_split;
+  p.out = static_cast<__half*>(out.ptr);
+  p.out_stride = out.row_stride;
+  float* ws = static_cast<float*>(workspace);
+  const size_t ws_rows = static_cast<size_t>(pl.kv_splits) * batch * n_heads * t_q;
+  p.ws_o = pl.kv_splits > 1 ? ws : nullptr;
+  p.ws_ml = pl.kv_splits > 1 ? ws + ws_rows * sea::fa::DH : nullptr;
+  p.err = dev->err;
+  p.limit_ns = sea::kDefaultTimeoutNs;
+
+  dim3 grid(ceil_div(pl.q_tiles, pl.nq) * pl.kv_splits, n_heads, batch);
+  if (pl.nq == 2) {
+    sea::fa::flash_attn_kernel<2>
+        <<<grid, sea::fa::Cfg<2>::THREADS, sea::fa::Cfg<2>::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  } else {
+    sea::fa::flash_attn_kernel<1>
+        <<<grid, sea::fa::Cfg<1>::THREADS, sea::fa::Cfg<1>::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  }
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  if (pl.kv_splits > 1) {
+    const int64_t rows = static_cast<int64_t>(batch) * n_heads * t_q;
+    sea::fa::combine_kernel<<<ceil_div(rows, 8), 256, 0, stream>>>(
+        p.ws_o, p.ws_ml, pl.kv_splits, batch, n_heads, t_q, p.out, p.out_stride);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+attn_status attn_qkv_pack(attn_mat x, const void* w_qkv, const void* b_q, const void* b_v, int64_t rows,
+                          int32_t d_model, attn_mat qkv_out, attn_stream_t stream) {
+  if (rows <= 0 || rows > INT32_MAX) return ATTN_ERR_INVALID;
+  if (d_model <= 0 || d_model % 64 != 0 || d_model > 65536) return ATTN_ERR_INVALID;
+  if (!valid_mat(x, d_model) || !valid_mat(qkv_out, 3 * static_cast<int64_t>(d_model))) return ATTN_ERR_INVALID;
+  if (w_qkv == nullptr || !aligned16(w_qkv)) return ATTN_ERR_INVALID;
+  if ((b_q != nullptr && !aligned16(b_q)) || (b_v != nullptr && !aligned16(b_v))) return ATTN_ERR_INVALID;
+  const int64_t n = 3 * static_cast<int64_t>(d_model);
+  const Range ro = mat_range(qkv_out.ptr, rows, n, qkv_out.row_stride);
+  if (overlaps(ro, mat_range(x.ptr, rows, d_model, x.row_stride)) ||
+      overlaps(ro, mat_range(w_qkv, n, d_model, d_model)))
+    return ATTN_ERR_INVALID;
+
+  DeviceInfo* dev = nullptr;
+  if (attn_status st = device_info(&dev); st != ATTN_OK) return st;
+
+  CUtensorMap tx, tw, to;
+  using namespace sea::gemm;
+  if (!encode_2d(&tx, x.ptr, d_model, rows, x.row_stride * 2, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&tw, w_qkv, d_model, n, static_cast<uint64_t>(d_model) * 2, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&to, qkv_out.ptr, n, rows, qkv_out.row_stride * 2, EPI_COLS, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+    return ATTN_ERR_CUDA;
+  Args a{};
+  a.b_q = static_cast<const __half*>(b_q);
+  a.b_v = static_cast<const __half*>(b_v);
+  a.m = static_cast<int>(rows);
+  a.n = static_cast<int>(n);
+  a.k = d_model;
+  a.d_model = d_model;
+  a.err = dev->err;
+  a.limit_ns = sea::kDefaultTimeoutNs;
+  const int64_t tiles = static_cast<int64_t>(ceil_div(rows, BM)) * ceil_div(n, BN);
+  const int grid = static_cast<int>(std::min<int64_t>(tiles, dev->num_sms));
+  qkv_gemm_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tx, tw, to, a);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  return ATTN_OK;
+}
+
+attn_status attn_forward(attn_mat q, attn_mat k, attn_mat v, int32_t batch, int32_t t_q, int32_t t_kv,
+                         int32_t n_heads, int32_t head_dim, attn_mask mask, float scale, attn_mat out,
+                         void* workspace, size_t workspace_bytes, attn_stream_t stream) {
+  return launch_attention(q, k, v, batch, t_q, t_kv, n_heads, head_dim, mask, scale, out, workspace,
+                          workspace_bytes, stream);
+}
+
+attn_status attn_cross(attn_mat q, attn_mat k_enc, attn_mat v_enc, int32_t batch, int32_t t_q, int32_t t_enc,
+                       int32_t n_heads, int32_t head_dim, float scale, attn_mat out, void* workspace,
+                       size_t workspace_bytes, attn_stream_t stream) {
+  attn_mask full{};
+  full.kind = ATTN_MASK_FULL;
+  return launch_attention(q, k_enc, v_enc, batch, t_q, t_enc, n_heads, head_dim, full, scale, out, workspace,
+                          workspace_bytes, stream);
+}
+
+size_t attn_workspace_size(int32_t batch, int32_t t_q, int32_t t_kv, int32_t n_heads, int32_t head_dim,
+                           int32_t mask_kind) {
+  if (batch <= 0 || t_q <= 0 || t_kv <= 0 || n_heads <= 0 || head_dim != sea::fa::DH) return 0;
+  if (mask_kind == ATTN_MASK_CHUNK) return 0;
+  DeviceInfo* dev = nullptr;
+  if (device_info(&dev) != ATTN_OK) return 0;
+  return plan_forward(batch, t_q, t_kv, n_heads, mask_kind, 0, dev->num_sms).ws_bytes;
+}
+
+const char* attn_status_string(attn_status status) {
+  switch (status) {
+    case ATTN_OK: return "ATTN_OK";
+    case ATTN_ERR_INVALID: return "ATTN_ERR_INVALID: invalid argument, nothing launched";
+    case ATTN_ERR_UNSUPPORTED: return "ATTN_ERR_UNSUPPORTED: needs an sm_100 (B200) device";
+    case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA: a CUDA call or kernel launch failed";
+    case ATTN_ERR_TIMEOUT: return "ATTN_ERR_TIMEOUT: a kernel's bounded wait expired";
+  }
+  return "ATTN_ERR_UNKNOWN";
+}
+
+attn_status attn_debug_error_word(attn_stream_t stream, uint32_t* word_out) {
+  DeviceInfo* dev = nullptr;
+  if (attn_status st = device_info(&dev); st != ATTN_OK) return st;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return ATTN_ERR_CUDA;
+  uint32_t w = 0;
+  if (cudaMemcpy(&w, dev->err, sizeof(w), cudaMemcpyDeviceToHost) != cudaSuccess) return ATTN_ERR_CUDA;
+  const uint32_t zero = 0;
+  if (cudaMemcpy(dev->err, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (word_out) *word_out = w;
+  return w ? ATTN_ERR_TIMEOUT : ATTN_OK;
+}
+
+attn_status attn_debug_timeout_probe(int64_t limit_ns, attn_stream_t stream) {
+  if (limit_ns < 1000 || limit_ns > 1000000000) return ATTN_ERR_INVALID;
+  DeviceInfo* dev = nullptr;
+  if (attn_status st = device_info(&dev); st != ATTN_OK) return st;
+  timeout_probe_kernel<<<1, 32, 0, stream>>>(dev->err, static_cast<uint64_t>(limit_ns));
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  return ATTN_OK;
+}
+
+}  // extern "C"

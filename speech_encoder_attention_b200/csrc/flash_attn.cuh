@@ -1,0 +1,508 @@
+// flash_attn.cuh -- fused multi-head flash attention on Blackwell tensor cores.
+//
+// Per head:  o_i = sum_{j in A_i} exp(s_ij - m_i) v_j / l_i,  s_ij = scale <q_i, k_j>
+// with the running max m and sum l kept in fp32 and no score matrix in memory.
+// The edda PR ("Add Edda ASR with DFlash2 speculative decoding", PR
+// description) replaces F32 scores materialised for all 1500 frames with flash
+// attention over F16 K/V; A_i is every key for the bidirectional encoder
+// window, the query's own chunk for the higgs chunked encoder
+// ("higgs-audio-v3-stt GGUF", "Architecture note (chunked encoder)"), and the
+// query row's ancestor slots for the token-tree verify pass (edda PR
+// description, beam search over a token-tree KV cache).
+//
+// One CTA owns NQ query tiles of 128 rows of one (sequence, head) and walks a
+// range of 128-row key/value tiles:
+//   warps [0, 4*NQ)  softmax: one thread per query row (tensor-memory lane ==
+//                    row, so a row's max and sum never leave the thread); the
+//                    same threads rescale O when the max grows and write the
+//                    normalised output.
+//   warp 4*NQ        TMA producer: Q once, then K and V tiles through a
+//                    3-stage ring, read in place from the (packed) projection
+//                    buffer through 3-D tensor maps (columns, frames, sequence),
+//                    so rows past a sequence's end read as zeros.
+//   warp 4*NQ+1      tcgen05.mma issuer: S = Q K^T (SS, 128x128x64) into tensor
+//                    memory, then O += P V (P from tensor memory, V MN-major in
+//                    shared memory, 128x64x128).
+// Tensor memory per query tile: S (128 fp32 columns), O (64), P (64 columns of
+// packed fp16 pairs).
+// Tile skipping: CHUNK walks only the key range of the query tile's chunk(s);
+// SLOTMASK skips key tiles whose mask words are zero for every row of the CTA.
+// Split-KV: for short query blocks the key range is split over CTAs; each
+// writes unnormalised O with its m and l to the workspace and a combine kernel
+// merges them.
+#pragma once
+
+#include "sm100_ptx.cuh"
+
+namespace sea {
+namespace fa {
+
+constexpr int BQ = 128;
+constexpr int BKV = 128;
+constexpr int DH = 64;
+constexpr int STAGES = 3;
+constexpr int TILE_BYTES = 128 * DH * 2;  // 16 KB, one 128-row x 64-col fp16 tile
+constexpr int MAX_FLAG_WORDS = 16;        // SLOTMASK: up to 512 key tiles (65536 slots)
+
+enum MaskKind : int { kFull = 0, kChunk = 1, kSlotmask = 2 };
+
+struct Params {
+  int batch, t_q, t_kv, n_heads;
+  float scale_log2;  // scale * log2(e)
+  int mask_kind;
+  int chunk_len;
+  const uint32_t* bits;
+  int words_per_row;
+  // query-tile schedule: the query axis is cut into segments of seg_len rows
+  // (whole chunks for CHUNK, the whole sequence otherwise), each segment into
+  // tiles_per_seg tiles of up to 128 rows.
+  int seg_len, tiles_per_seg, q_tiles;
+  // key/value split
+  int kv_splits, kv_tiles_per_split;
+  // outputs
+  __half* out;
+  int64_t out_stride;
+  float* ws_o;   // [splits][batch][heads][t_q][64] unnormalised partial O
+  float* ws_ml;  // [splits][batch][heads][t_q][2]  (m in log2 units, l)
+  uint32_t* err;
+  uint64_t limit_ns;
+};
+
+template <int NQ>
+struct Cfg {
+  static constexpr int SOFTMAX_THREADS = 128 * NQ;
+  static constexpr int THREADS = SOFTMAX_THREADS + 64;
+  static constexpr int PRODUCER_WARP = 4 * NQ;
+  static constexpr int MMA_WARP = 4 * NQ + 1;
+  static constexpr int TMEM_COLS = NQ == 1 ? 256 : 512;
+  __host__ __device__ static constexpr uint32_t S_COL(int q) { return 128u * q; }
+  __host__ __device__ static constexpr uint32_t O_COL(int q) { return 128u * NQ + 64u * q; }
+  __host__ __device__ static constexpr uint32_t P_COL(int q) { return 128u * NQ + 64u * NQ + 64u * q; }
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + NQ * TILE_BYTES;
+  static constexpr int OFF_V = OFF_K + STAGES * TILE_BYTES;
+  static constexpr int OFF_BARS = OFF_V + STAGES * TILE_BYTES;
+  // q_full, k_full[S], v_full[S], kv_empty[S], s_full[NQ], s_free[NQ], p_full[NQ], o_done[NQ], drain
+  static constexpr int NUM_BARS = 1 + 3 * STAGES + 4 * NQ + 1;
+  static constexpr int OFF_FLAGS = OFF_BARS + 8 * NUM_BARS;
+  static constexpr int OFF_MISC = OFF_FLAGS + 4 * MAX_FLAG_WORDS;
+  static constexpr int SMEM_BYTES = 1024 + OFF_MISC + 16;
+};
+
+struct TileGeom {
+  int q0;     // first query row (sequence-local)
+  int rows;   // valid rows in the tile (0 if none)
+};
+
+__device__ __forceinline__ TileGeom q_tile_geom(const Params& p, int qt) {
+  TileGeom g{p.t_q, 0};
+  if (qt >= p.q_tiles) return g;
+  const int seg = qt / p.tiles_per_seg;
+  const int w = qt - seg * p.tiles_per_seg;
+  const int seg0 = seg * p.seg_len;
+  const int q0 = seg0 + w * BQ;
+  const int seg_end = min(seg0 + p.seg_len, p.t_q);
+  g.q0 = q0;
+  g.rows = max(0, min(BQ, seg_end - q0));
+  if (g.rows == 0) g.q0 = p.t_q;
+  return g;
+}
+
+template <int NQ>
+__global__ void __launch_bounds__(Cfg<NQ>::THREADS, 1)
+    flash_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const Params p) {
+  using C = Cfg<NQ>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + C::OFF_BARS;
+  const uint32_t q_full = bar0;
+  auto k_full = [&](int s) { return bar0 + 8u * (1 + s); };
+  auto v_full = [&](int s) { return bar0 + 8u * (1 + STAGES + s); };
+  auto kv_empty = [&](int s) { return bar0 + 8u * (1 + 2 * STAGES + s); };
+  auto s_full = [&](int q) { return bar0 + 8u * (1 + 3 * STAGES + q); };
+  auto s_free = [&](int q) { return bar0 + 8u * (1 + 3 * STAGES + NQ + q); };
+  auto p_full = [&](int q) { return bar0 + 8u * (1 + 3 * STAGES + 2 * NQ + q); };
+  auto o_done = [&](int q) { return bar0 + 8u * (1 + 3 * STAGES + 3 * NQ + q); };
+  const uint32_t drain_bar = bar0 + 8u * (1 + 3 * STAGES + 4 * NQ);
+  uint32_t* flags = reinterpret_cast<uint32_t*>(smem + C::OFF_FLAGS);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + C::OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int split = blockIdx.x % p.kv_splits;
+  const int qgroup = blockIdx.x / p.kv_splits;
+  const int h = blockIdx.y;
+  const int b = blockIdx.z;
+
+  // Query tiles of this CTA and the key range they need.
+  TileGeom geom[NQ];
+  int any_rows = 0;
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) {
+    geom[q] = q_tile_geom(p, qgroup * NQ + q);
+    any_rows |= geom[q].rows;
+  }
+  if (!any_rows) return;  // uniform for the whole CTA: nothing allocated yet
+
+  int kv_lo = 0, kv_hi = p.t_kv;
+  if (p.mask_kind == kChunk) {
+    int lo = INT_MAX, hi = 0;
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+      if (geom[q].rows == 0) continue;
+      lo = min(lo, (geom[q].q0 / p.chunk_len) * p.chunk_len);
+      const int last = geom[q].q0 + geom[q].rows - 1;
+      hi = max(hi, min((last / p.chunk_len + 1) * p.chunk_len, p.t_kv));
+    }
+    kv_lo = lo;
+    kv_hi = hi;
+  }
+  const int n_kv = (kv_hi - kv_lo + BKV - 1) / BKV;
+  const int j_begin = min(n_kv, split * p.kv_tiles_per_split);
+  const int j_end = min(n_kv, j_begin + p.kv_tiles_per_split);
+  const bool use_flags = p.mask_kind == kSlotmask;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(k_full(s), 1);
+      mbar_init(v_full(s), 1);
+      mbar_init(kv_empty(s), 1);
+    }
+    for (int q = 0; q < NQ; ++q) {
+      mbar_init(s_full(q), 1);
+      mbar_init(s_free(q), 4);
+      mbar_init(p_full(q), 4);
+      mbar_init(o_done(q), 1);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0u;
+    fence_barrier_init();
+  }
+  if (threadIdx.x < MAX_FLAG_WORDS) flags[threadIdx.x] = 0u;
+  if (warp == C::MMA_WARP) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const WaitCtl wc{abort_flag, p.err, p.limit_ns};
+
+  // Softmax-thread identity (meaningful for threadIdx.x < SOFTMAX_THREADS).
+  const int sq = threadIdx.x >> 7;          // query tile of this thread
+  const int srow = threadIdx.x & 127;       // row within the tile == TMEM lane
+  const int qsel = sq < NQ ? sq : 0;
+  const int row_glob = geom[qsel].q0 + srow;  // sequence-local query row
+  const bool row_ok = threadIdx.x < C::SOFTMAX_THREADS && srow < geom[qsel].rows;
+  const uint32_t* mask_row =
+      (use_flags && row_ok) ? p.bits + static_cast<int64_t>(row_glob) * p.words_per_row : nullptr;
+
+  // SLOTMASK: mark key tiles that any row of this CTA may see.
+  if (use_flags) {
+    if (mask_row != nullptr) {
+      for (int j = j_begin; j < j_end; ++j) {
+        const int w0 = j * (BKV / 32);
+        uint32_t any = 0;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (w0 + c < p.words_per_row) any |= __ldg(mask_row + w0 + c);
+        if (any) atomicOr(&flags[j >> 5], 1u << (j & 31));
+      }
+    }
+    __syncthreads();
+  }
+  auto tile_on = [&](int j) -> bool { return !use_flags || ((flags[j >> 5] >> (j & 31)) & 1u); };
+
+  if (warp == C::PRODUCER_WARP) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(q_full, NQ * TILE_BYTES);
+#pragma unroll
+      for (int q = 0; q < NQ; ++q)
+        tma_load_3d(sbase + C::OFF_Q + q * TILE_BYTES, &tm_q, q_full, h * DH, geom[q].q0, b);
+      int it = 0;
+      for (int j = j_begin; j < j_end; ++j) {
+        if (!tile_on(j)) continue;
+        const int st = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        if (!mbar_wait(kv_empty(st), ph ^ 1u, wc)) break;
+        const int kv0 = kv_lo + j * BKV;
+        mbar_arrive_expect_tx(k_full(st), TILE_BYTES);
+        tma_load_3d(sbase + C::OFF_K + st * TILE_BYTES, &tm_k, k_full(st), h * DH, kv0, b);
+        mbar_arrive_expect_tx(v_full(st), TILE_BYTES);
+        tma_load_3d(sbase + C::OFF_V + st * TILE_BYTES, &tm_v, v_full(st), h * DH, kv0, b);
+        ++it;
+      }
+      // Let the copies land before the CTA may exit.
+      mbar_wait_drain(q_full, 0, p.limit_ns);
+      for (int i = max(0, it - STAGES); i < it; ++i) {
+        mbar_wait_drain(k_full(i % STAGES), (i / STAGES) & 1, p.limit_ns);
+        mbar_wait_drain(v_full(i % STAGES), (i / STAGES) & 1, p.limit_ns);
+      }
+    }
+  } else if (warp == C::MMA_WARP) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      constexpr uint32_t idesc_s = idesc_f16_f32(BQ, BKV, 0, 0);  // Q, K both K-major
+      constexpr uint32_t idesc_o = idesc_f16_f32(BQ, DH, 0, 1);   // P K-major (TMEM), V MN-major
+      bool ok = mbar_wait(q_full, 0, wc);
+      int it = 0;
+      int prev_st = 0;
+      auto issue_pv = [&](int st, int idx) -> bool {
+        if (!mbar_wait(v_full(st), (idx / STAGES) & 1, wc)) return false;
+        const uint32_t sv = sbase + C::OFF_V + st * TILE_BYTES;
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) {
+          if (!mbar_wait(p_full(q), idx & 1, wc)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < BKV / 16; ++kk) {
+            const uint64_t vd = smem_desc_sw128(sv + kk * 2048, TILE_BYTES, 1024);
+            mma_f16_ts(tmem_base + C::O_COL(q), tmem_base + C::P_COL(q) + kk * 8, vd, idesc_o,
+                       (idx > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(o_done(q));
+        }
+        mma_commit(kv_empty(st));
+        return true;
+      };
+      for (int j = j_begin; j < j_end && ok; ++j) {
+        if (!tile_on(j)) continue;
+        const int st = it % STAGES;
+        if (!mbar_wait(k_full(st), (it / STAGES) & 1, wc)) {
+          ok = false;
+          break;
+        }
+        const uint32_t sk = sbase + C::OFF_K + st * TILE_BYTES;
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) {
+          if (it > 0 && !mbar_wait(s_free(q), (it - 1) & 1, wc)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sq_addr = sbase + C::OFF_Q + q * TILE_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < DH / 16; ++kk) {
+            const uint64_t qd = smem_desc_sw128(sq_addr + kk * 32, 16, 1024);
+            const uint64_t kd = smem_desc_sw128(sk + kk * 32, 16, 1024);
+            mma_f16_ss(tmem_base + C::S_COL(q), qd, kd, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(s_full(q));
+        }
+        if (!ok) break;
+        if (it > 0 && !issue_pv(prev_st, it - 1)) {
+          ok = false;
+          break;
+        }
+        prev_st = st;
+        ++it;
+      }
+      if (ok && it > 0) issue_pv(prev_st, it - 1);
+      mma_commit(drain_bar);
+      mbar_wait_drain(drain_bar, 0, p.limit_ns);
+    }
+  } else {
+    // ---------------- softmax / correction / epilogue ----------------
+    const int q = sq;
+    const uint32_t lane_field = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t s_tmem = tmem_base + C::S_COL(q) + lane_field;
+    const uint32_t o_tmem = tmem_base + C::O_COL(q) + lane_field;
+    const uint32_t p_tmem = tmem_base + C::P_COL(q) + lane_field;
+    // Allowed key range of this row for FULL / CHUNK (sequence-local indices).
+    int lo_i = 0, hi_i = p.t_kv;
+    if (p.mask_kind == kChunk) {
+      lo_i = (row_glob / p.chunk_len) * p.chunk_len;
+      hi_i = min(lo_i + p.chunk_len, p.t_kv);
+    }
+    if (!row_ok) {
+      lo_i = 0;
+      hi_i = 0;
+    }
+    const float sl2 = p.scale_log2;
+    float m_run = -INFINITY;
+    float l_run = 0.f;
+    int it = 0;
+    bool ok = true;
+    for (int j = j_begin; j < j_end; ++j) {
+      if (!tile_on(j)) continue;
+      if (!mbar_wait(s_full(q), it & 1, wc)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float s[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(s_tmem + c * 32, r);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(r[e]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free(q));
+
+      const int kv0 = kv_lo + j * BKV;
+      if (use_flags) {
+        uint32_t wbits[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int wi = (kv0 >> 5) + c;
+          wbits[c] = (mask_row != nullptr && wi < p.words_per_row) ? __ldg(mask_row + wi) : 0u;
+        }
+        const int lim = p.t_kv - kv0;
+#pragma unroll
+        for (int e = 0; e < 128; ++e)
+          if (!((wbits[e >> 5] >> (e & 31)) & 1u) || e >= lim) s[e] = -INFINITY;
+      } else {
+        const int a = lo_i - kv0;
+        const int bnd = hi_i - kv0;
+        if (a > 0 || bnd < BKV) {
+#pragma unroll
+          for (int e = 0; e < 128; ++e)
+            if (e < a || e >= bnd) s[e] = -INFINITY;
+        }
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int e = 1; e < 128; ++e) mx = fmaxf(mx, s[e]);
+      const float m_new = fmaxf(m_run, mx * sl2);
+      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+      const float alpha = ex2_approx(m_run - m_use);
+      float sum = 0.f;
+      uint32_t pk[64];
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        const float p0 = ex2_approx(fmaf(s[2 * i], sl2, -m_use));
+        const float p1 = ex2_approx(fmaf(s[2 * i + 1], sl2, -m_use));
+        sum += p0 + p1;
+        pk[i] = pack_half2(p0, p1);
+      }
+      l_run = l_run * alpha + sum;
+      if (it > 0) {
+        if (!mbar_wait(o_done(q), (it - 1) & 1, wc)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            uint32_t r[32];
+            tmem_ld32(o_tmem + c * 32, r);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+            tmem_st32(o_tmem + c * 32, r);
+          }
+        }
+      }
+      {
+        uint32_t r0[32], r1[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          r0[e] = pk[e];
+          r1[e] = pk[32 + e];
+        }
+        tmem_st32(p_tmem, r0);
+        tmem_st32(p_tmem + 32, r1);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full(q));
+      m_run = m_new;
+      ++it;
+    }
+
+    // ---------------- epilogue ----------------
+    float o[64];
+#pragma unroll
+    for (int e = 0; e < 64; ++e) o[e] = 0.f;
+    if (ok && it > 0 && mbar_wait(o_done(q), (it - 1) & 1, wc)) {
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t r[32];
+        tmem_ld32(o_tmem + c * 32, r);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[c * 32 + e] = __uint_as_float(r[e]);
+      }
+    }
+    if (row_ok) {
+      if (p.kv_splits > 1) {
+        const int64_t idx =
+            ((static_cast<int64_t>(split) * p.batch + b) * p.n_heads + h) * p.t_q + row_glob;
+        float4* dst = reinterpret_cast<float4*>(p.ws_o + idx * DH);
+#pragma unroll
+        for (int v = 0; v < 16; ++v) dst[v] = make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+        reinterpret_cast<float2*>(p.ws_ml)[idx] = make_float2(m_run, l_run);
+      } else {
+        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+        __half* dst = p.out + (static_cast<int64_t>(b) * p.t_q + row_glob) * p.out_stride + h * DH;
+        uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          uint4 u;
+          u.x = pack_half2(o[8 * v + 0] * inv, o[8 * v + 1] * inv);
+          u.y = pack_half2(o[8 * v + 2] * inv, o[8 * v + 3] * inv);
+          u.z = pack_half2(o[8 * v + 4] * inv, o[8 * v + 5] * inv);
+          u.w = pack_half2(o[8 * v + 6] * inv, o[8 * v + 7] * inv);
+          d4[v] = u;
+        }
+      }
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == C::MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// Merges the split-KV partials of one (sequence, head, row) per warp:
+//   M = max_s m_s,  L = sum_s l_s 2^(m_s - M),  o = sum_s O_s 2^(m_s - M) / L.
+__global__ void __launch_bounds__(256)
+    combine_kernel(const float* __restrict__ ws_o, const float* __restrict__ ws_ml, int splits,
+                   int batch, int n_heads, int t_q, __half* __restrict__ out, int64_t out_stride) {
+  const int64_t rows = static_cast<int64_t>(batch) * n_heads * t_q;
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (idx >= rows) return;
+  const int lane = threadIdx.x & 31;
+  const int r = static_cast<int>(idx % t_q);
+  const int h = static_cast<int>((idx / t_q) % n_heads);
+  const int b = static_cast<int>(idx / (static_cast<int64_t>(t_q) * n_heads));
+  const int64_t stride = rows;  // entries between consecutive splits
+  float mmax = -INFINITY;
+  for (int s = 0; s < splits; ++s) {
+    const float2 ml = reinterpret_cast<const float2*>(ws_ml)[idx + s * stride];
+    if (ml.y > 0.f) mmax = fmaxf(mmax, ml.x);
+  }
+  float l = 0.f, o0 = 0.f, o1 = 0.f;
+  if (mmax != -INFINITY) {
+    for (int s = 0; s < splits; ++s) {
+      const float2 ml = reinterpret_cast<const float2*>(ws_ml)[idx + s * stride];
+      if (!(ml.y > 0.f)) continue;
+      const float w = ex2_approx(ml.x - mmax);
+      l += ml.y * w;
+      const float2 ov = reinterpret_cast<const float2*>(ws_o + (idx + s * stride) * DH)[lane];
+      o0 += ov.x * w;
+      o1 += ov.y * w;
+    }
+  }
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+  __half2* dst = reinterpret_cast<__half2*>(out + (static_cast<int64_t>(b) * t_q + r) * out_stride + h * DH);
+  dst[lane] = __floats2half2_rn(o0 * inv, o1 * inv);
+}
+
+}  // namespace fa
+}  // namespace sea

@@ -1,0 +1,271 @@
+// qkv_gemm.cuh -- the packed QKV projection on Blackwell tensor cores.
+//
+//   qkv[r, j] = sum_c x[r, c] * W[j, c] + bias[j],   bias = [b_q | 0 | b_v]
+//
+// The edda PR ("Add Edda ASR with DFlash2 speculative decoding", PR
+// description) packs the three projections into one; this is that single GEMM
+// with the q/v bias folded into its epilogue (Whisper's key projection has no
+// bias).
+//
+// Design (one persistent CTA per SM, 192 threads):
+//   warp 0      TMA producer: x and W tiles (64-wide K slices, 128-byte swizzle)
+//               into a 4-stage shared-memory ring.
+//   warp 1      tcgen05.mma issuer (one thread): 128x256x16 f16 MMAs into one of
+//               two 256-column fp32 accumulators in tensor memory, so the
+//               epilogue of tile i overlaps the main loop of tile i+1.
+//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, add the bias in fp32,
+//               round to fp16, stage a 32x32 box per warp in swizzled shared
+//               memory and write it with a TMA store.
+// Both operands are K-major (x rows and W rows are contiguous along d_model).
+#pragma once
+
+#include "sm100_ptx.cuh"
+
+namespace sea {
+namespace gemm {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;
+constexpr int STAGES = 4;
+constexpr int EPI_COLS = 32;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BN * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int EPI_BUF_BYTES = 32 * EPI_COLS * 2;  // one 32-row x 32-col fp16 box
+constexpr int EPI_BYTES = 4 * 2 * EPI_BUF_BYTES;  // 4 warps, double buffered
+constexpr int THREADS = 192;
+constexpr int TMEM_COLS = 512;  // two accumulators of BN fp32 columns
+
+constexpr int OFF_STAGES = 0;
+constexpr int OFF_EPI = OFF_STAGES + STAGES * STAGE_BYTES;
+constexpr int OFF_BARS = OFF_EPI + EPI_BYTES;
+// barriers: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain
+constexpr int NUM_BARS = 2 * STAGES + 5;
+constexpr int OFF_MISC = OFF_BARS + 8 * NUM_BARS;  // tmem base, abort flag
+constexpr int SMEM_BYTES = 1024 + OFF_MISC + 16;   // + slack to align the base to 1 KB
+
+struct Args {
+  const __half* b_q;
+  const __half* b_v;
+  int m, n, k, d_model;
+  uint32_t* err;
+  uint64_t limit_ns;
+};
+
+__device__ __forceinline__ void load_bias32(const Args& a, int n_c, float (&bias)[32]) {
+  const __half* src = nullptr;
+  const int region = n_c / a.d_model;
+  if (region == 0)
+    src = a.b_q ? a.b_q + n_c : nullptr;
+  else if (region == 2)
+    src = a.b_v ? a.b_v + (n_c - 2 * a.d_model) : nullptr;
+  if (src == nullptr) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) bias[i] = 0.f;
+    return;
+  }
+  const uint4* s4 = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    uint4 u = __ldg(s4 + v);
+    const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 f = __half22float2(h[i]);
+      bias[8 * v + 2 * i] = f.x;
+      bias[8 * v + 2 * i + 1] = f.y;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    qkv_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                    const __grid_constant__ CUtensorMap tm_out, const Args args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + OFF_BARS;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int tiles_m = (args.m + BM - 1) / BM;
+  const int tiles_n = (args.n + BN - 1) / BN;
+  const int num_tiles = tiles_m * tiles_n;
+  const int kblocks = (args.k + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 4);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0u;
+    fence_barrier_init();
+    tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_w);
+    tma_prefetch_desc(&tm_out);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const WaitCtl wc{abort_flag, args.err, args.limit_ns};
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+        const int m0 = (tile / tiles_n) * BM;
+        const int n0 = (tile % tiles_n) * BN;
+        bool ok = true;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, wc)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sa = sbase + OFF_STAGES + stage * STAGE_BYTES;
+          mbar_arrive_expect_tx(full_bar(stage), STAGE_BYTES);
+          tma_load_2d(sa, &tm_x, full_bar(stage), kb * BK, m0);
+          tma_load_2d(sa + A_BYTES, &tm_w, full_bar(stage), kb * BK, n0);
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+      }
+      // Let the last copies land before the CTA can exit (they are already
+      // complete on the normal path).
+      for (int i = 0; i < STAGES && i < issued; ++i) {
+        if (--stage < 0) {
+          stage = STAGES - 1;
+          phase ^= 1u;
+        }
+        mbar_wait_drain(full_bar(stage), phase, args.limit_ns);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      constexpr uint32_t idesc = idesc_f16_f32(BM, BN, 0, 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
+        const int acc = local & 1;
+        const uint32_t acc_phase = (local >> 1) & 1;
+        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, wc)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, wc)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = sbase + OFF_STAGES + stage * STAGE_BYTES;
+          const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = smem_desc_sw128(sa + kk * 32, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(sb + kk * 32, 16, 1024);
+            mma_f16_ss(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          mma_commit(empty_bar(stage));
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (ok) mma_commit(tfull_bar(acc));
+      }
+      // Every MMA issued above has finished once this arrives.
+      mma_commit(drain_bar);
+      mbar_wait_drain(drain_bar, 0, args.limit_ns);
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int quad = warp & 3;  // tensor-memory lane quadrant this warp may access
+    const uint32_t lane_field = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t ebuf = sbase + OFF_EPI + (warp - 2) * 2 * EPI_BUF_BYTES;
+    uint32_t chunk_count = 0;
+    int local = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      if (!mbar_wait(tfull_bar(acc), acc_phase, wc)) break;
+      tc_fence_after();
+      const int m0 = (tile / tiles_n) * BM;
+      const int n0 = (tile % tiles_n) * BN;
+      const int row0 = m0 + quad * 32;
+#pragma unroll 1
+      for (int c = 0; c < BN / EPI_COLS; ++c) {
+        const int n_c = n0 + c * EPI_COLS;
+        if (n_c >= args.n) break;
+        uint32_t r[32];
+        tmem_ld32(tmem_base + acc * BN + c * EPI_COLS + lane_field, r);
+        float bias[32];
+        load_bias32(args, n_c, bias);
+        uint32_t h[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          h[i] = pack_half2(__uint_as_float(r[2 * i]) + bias[2 * i],
+                            __uint_as_float(r[2 * i + 1]) + bias[2 * i + 1]);
+        const uint32_t buf = ebuf + (chunk_count & 1u) * EPI_BUF_BYTES;
+        if (lane == 0) bulk_wait_group_read<1>();
+        __syncwarp();
+        // Row `lane` of the 32x32 box, 64 bytes, in the 64-byte swizzle TMA expects.
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const uint32_t addr = buf + lane * 64 + ((v ^ ((lane >> 1) & 3)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(h[4 * v]),
+                       "r"(h[4 * v + 1]), "r"(h[4 * v + 2]), "r"(h[4 * v + 3])
+                       : "memory");
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && row0 < args.m) {
+          tma_store_2d(&tm_out, buf, n_c, row0);
+          bulk_commit_group();
+        }
+        ++chunk_count;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty_bar(acc));
+    }
+    if (lane == 0) bulk_wait_group_all();
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace gemm
+}  // namespace sea
