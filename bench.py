@@ -1,0 +1,587 @@
+#!/usr/bin/env python3
+"""Benchmark of the Whisper-style attention pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload windows8]
+    python bench.py --impl reference ...      # the FP64 CPU oracle on host cores
+
+One step = the whole hot path over one batch: the packed QKV projection
+(attn_qkv_pack) followed by multi-head flash attention (attn_forward), for the
+8-window encoder workload (8 x 1500 frames, d_model 1280, 20 heads of 64, FULL
+mask). Inputs are resident in HBM when the timed region starts; L2 is flushed
+(a 256 MiB write) between timed steps, outside the per-step CUDA events. Every
+launch is timed with CUDA events on the stream it runs on. With N > 1 (one
+process per GPU under torchrun) each rank runs its own 8 windows (weak
+scaling, no collective on the data path) and the step time is the maximum
+over ranks.
+
+Rank 0 prints one JSON line. `value` is the whole-job throughput in TFLOP/s of
+algorithmic QKV + attention flops; `e2e` is the same metric through the same C
+ABI calls with the step's input copied from pinned host memory and its output
+copied back inside the timed region.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import socket
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from speech_encoder_attention_b200 import inputs  # noqa: E402
+
+METRIC = "attention+QKV TFLOP/s at T=1500, 20x64 heads; % of B200 FP16 tensor peak"
+FLUSH_BYTES = 256 << 20
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+KERNEL_SOURCES = ["speech_encoder_attention_b200/csrc/flash_attn.cuh",
+                  "speech_encoder_attention_b200/csrc/qkv_gemm.cuh",
+                  "speech_encoder_attention_b200/csrc/sm100_ptx.cuh",
+                  "speech_encoder_attention_b200/csrc/attn_api.cu"]
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work
+# ---------------------------------------------------------------------------
+
+def qkv_flops(rows: int, d: int) -> float:
+    return 2.0 * rows * d * 3 * d
+
+
+def attn_pair_flops(pairs: int, heads: int, dh: int = 64) -> float:
+    """2*dh flops for the score and 2*dh for the value product, per allowed pair and head."""
+    return 4.0 * dh * heads * pairs
+
+
+def encoder_pairs(spec: inputs.EncoderSpec) -> int:
+    if spec.mask == "chunk":
+        full, rest = divmod(spec.t, spec.chunk_len)
+        return spec.batch * (full * spec.chunk_len ** 2 + rest ** 2)
+    return spec.batch * spec.t * spec.t
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    if os.path.exists(PEAKS_FILE):
+        with open(PEAKS_FILE) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def stored_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            doc = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = doc.get(workload, {}).get(kernel)
+    if not ent or ent.get("source_hash") != kernel_source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only)
+# ---------------------------------------------------------------------------
+
+REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.period = period_s
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._nvml = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nvml = None
+
+    def _run(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                util = nv.nvmlDeviceGetUtilizationRates(self._h).gpu
+                try:
+                    reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                except AttributeError:
+                    reasons = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+                self.samples.append((sm, util, reasons))
+            except Exception:
+                pass
+            self._stop.wait(self.period)
+
+    def __enter__(self):
+        if self._nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "note": "no NVML samples"}
+        loaded = [s for s in self.samples if s[1] > 0] or self.samples
+        mhz = sorted(s[0] for s in loaded)
+        bits = 0
+        for s in loaded:
+            bits |= int(s[2])
+        reasons = [name for bit, name in REASON_BITS.items() if bits & bit and name != "gpu_idle"]
+        return {"sm_mhz": mhz[len(mhz) // 2], "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(self.samples), "samples_under_load": len(loaded)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (host side; covered by CPU gloo tests)
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def reduce_step_time(local_ms: float, device=None) -> float:
+    """Max of the per-rank device-timed step time over all ranks."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return local_ms
+    t = torch.tensor([local_ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank_step: float, world: int, ms_per_step: float) -> float:
+    """Units all ranks processed per second, at the slowest rank's step time."""
+    return units_per_rank_step * world / (ms_per_step * 1e-3)
+
+
+def relaunch_under_torchrun(n: int, argv):
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
+
+
+# ---------------------------------------------------------------------------
+# workloads on the GPU
+# ---------------------------------------------------------------------------
+
+class EncoderStep:
+    """Packed projection + attention over a batch of windows (or chunks)."""
+
+    def __init__(self, spec: inputs.EncoderSpec, device):
+        import torch
+        from speech_encoder_attention_b200 import attn
+        self.attn = attn
+        self.spec = spec
+        inp = inputs.make_encoder_inputs(spec)
+        dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+        self.x, self.w, self.bq, self.bv = dev(inp.x), dev(inp.w_qkv), dev(inp.b_q), dev(inp.b_v)
+        rows, d = inp.x.shape
+        self.d = d
+        self.qkv = torch.empty(rows, 3 * d, dtype=torch.float16, device=device)
+        self.out = torch.empty(rows, d, dtype=torch.float16, device=device)
+        self.mask = attn.MASK_CHUNK if spec.mask == "chunk" else attn.MASK_FULL
+        self.host_x = torch.from_numpy(inp.x).pin_memory()
+        self.host_out = torch.empty(rows, d, dtype=torch.float16).pin_memory()
+        self.kernels = ["qkv_gemm", "flash_attn"]
+        self.flops = {"qkv_gemm": qkv_flops(rows, d),
+                      "flash_attn": attn_pair_flops(encoder_pairs(spec), spec.n_heads)}
+        self.launches_per_step = 2
+
+    def run(self, events=None):
+        a, d, s = self.attn, self.d, self.spec
+        if events:
+            events[0].record()
+        a.attn_qkv_pack(self.x, self.w, self.bq, self.bv, out=self.qkv)
+        if events:
+            events[1].record()
+        a.attn_forward(self.qkv[:, :d], self.qkv[:, d:2 * d], self.qkv[:, 2 * d:], s.batch, s.t, s.t, s.n_heads,
+                       mask_kind=self.mask, chunk_len=s.chunk_len, out=self.out, split=False)
+        if events:
+            events[2].record()
+
+    def run_e2e(self, events=None):
+        if events:
+            events[0].record()
+        self.x.copy_(self.host_x, non_blocking=True)
+        self.run()
+        self.host_out.copy_(self.out, non_blocking=True)
+        if events:
+            events[-1].record()
+
+    @property
+    def h2d_bytes(self):
+        return self.host_x.numel() * 2
+
+    @property
+    def d2h_bytes(self):
+        return self.host_out.numel() * 2
+
+    def total_flops(self):
+        return sum(self.flops.values())
+
+    def units(self):
+        return {"frames": self.spec.batch * self.spec.t}
+
+
+class VerifyStep:
+    """Token-tree self-attention (SLOTMASK) plus cross-attention of the same block."""
+
+    def __init__(self, spec: inputs.VerifySpec, device):
+        import torch
+        from speech_encoder_attention_b200 import attn
+        self.attn = attn
+        self.spec = spec
+        inp = inputs.make_verify_inputs(spec)
+        dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+        self.q, self.kc, self.vc = dev(inp.q), dev(inp.k_cache), dev(inp.v_cache)
+        self.ke, self.ve = dev(inp.k_enc), dev(inp.v_enc)
+        self.bits = dev(inp.bits.view(np.int32))
+        d = spec.d_model
+        self.o_self = torch.empty(spec.t_q, d, dtype=torch.float16, device=device)
+        self.o_cross = torch.empty(spec.t_q, d, dtype=torch.float16, device=device)
+        ws = max(attn.workspace_size(1, spec.t_q, spec.slots, spec.n_heads, attn.MASK_SLOTMASK),
+                 attn.workspace_size(1, spec.t_q, spec.t_enc, spec.n_heads, attn.MASK_FULL))
+        self.ws = torch.empty(max(ws, 16), dtype=torch.uint8, device=device)
+        self.host_q = torch.from_numpy(inp.q).pin_memory()
+        self.host_out = torch.empty(2 * spec.t_q, d, dtype=torch.float16).pin_memory()
+        pairs = int(inputs.unpack_bits(inp.bits, spec.slots).sum())
+        self.kernels = ["slotmask_attn", "cross_attn"]
+        self.flops = {"slotmask_attn": attn_pair_flops(pairs, spec.n_heads),
+                      "cross_attn": attn_pair_flops(spec.t_q * spec.t_enc, spec.n_heads)}
+        b = 2
+        self.bytes = {
+            "slotmask_attn": b * d * (spec.t_q + 2 * spec.slots + spec.t_q) + 4 * inp.bits.size,
+            "cross_attn": b * d * (spec.t_q + 2 * spec.t_enc + spec.t_q),
+        }
+        self.launches_per_step = 4  # two attention kernels, each followed by its split combine
+
+    def run(self, events=None):
+        a, s = self.attn, self.spec
+        if events:
+            events[0].record()
+        a.attn_forward(self.q, self.kc, self.vc, 1, s.t_q, s.slots, s.n_heads, mask_kind=a.MASK_SLOTMASK,
+                       bits=self.bits, out=self.o_self, workspace=self.ws)
+        if events:
+            events[1].record()
+        a.attn_cross(self.q, self.ke, self.ve, 1, s.t_q, s.t_enc, s.n_heads, out=self.o_cross, workspace=self.ws)
+        if events:
+            events[2].record()
+
+    def run_e2e(self, events=None):
+        if events:
+            events[0].record()
+        self.q.copy_(self.host_q, non_blocking=True)
+        self.run()
+        self.host_out[:self.spec.t_q].copy_(self.o_self, non_blocking=True)
+        self.host_out[self.spec.t_q:].copy_(self.o_cross, non_blocking=True)
+        if events:
+            events[-1].record()
+
+    @property
+    def h2d_bytes(self):
+        return self.host_q.numel() * 2
+
+    @property
+    def d2h_bytes(self):
+        return self.host_out.numel() * 2
+
+    def total_flops(self):
+        return sum(self.flops.values())
+
+    def total_bytes(self):
+        return sum(self.bytes.values())
+
+    def units(self):
+        return {"query_rows": self.spec.t_q}
+
+
+def make_step(name, device):
+    if name in inputs.ENCODER_WORKLOADS:
+        return EncoderStep(inputs.ENCODER_WORKLOADS[name], device)
+    return VerifyStep(inputs.VERIFY_WORKLOADS[name], device)
+
+
+# ---------------------------------------------------------------------------
+# oracle timing (host cores): the reference arm and the cpu_baseline leg
+# ---------------------------------------------------------------------------
+
+def oracle_sample(spec: inputs.EncoderSpec, inp, i: int):
+    """One bounded sample of the encoder workload: window i % batch, head
+    i % n_heads -- that head's slice of the packed projection (q, k, v columns)
+    and its attention over the window, by the FP64 oracle. Returns flops."""
+    import oracle
+    d, t = spec.d_model, spec.t
+    b, h = i % spec.batch, i % spec.n_heads
+    cols = np.r_[h * 64:(h + 1) * 64, d + h * 64:d + (h + 1) * 64, 2 * d + h * 64:2 * d + (h + 1) * 64]
+    x = inp.x[b * t:(b + 1) * t]
+    qkv = oracle.qkv_projection(x, inp.w_qkv[cols], inp.b_q[h * 64:(h + 1) * 64], inp.b_v[h * 64:(h + 1) * 64])
+    allowed = oracle.allowed_full(t, t) if spec.mask == "full" else oracle.allowed_chunk(t, spec.chunk_len)
+    oracle.attention(qkv[:, :64], qkv[:, 64:128], qkv[:, 128:], 1, allowed)
+    pairs = encoder_pairs(inputs.EncoderSpec("s", 1, t, d, 1, spec.mask, spec.chunk_len, 0))
+    return 2.0 * t * d * 192 + attn_pair_flops(pairs, 1)
+
+
+def oracle_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info()]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def time_oracle(spec, seconds: float = 10.0, max_samples: int = 400):
+    inp = inputs.make_encoder_inputs(spec)
+    oracle_sample(spec, inp, 0)  # warm
+    t0 = time.perf_counter()
+    flops, n = 0.0, 0
+    while n < max_samples and (time.perf_counter() - t0 < seconds or n == 0):
+        flops += oracle_sample(spec, inp, n)
+        n += 1
+    el = time.perf_counter() - t0
+    return {"value": flops / el / 1e12, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"{n} samples of (one window x one head) of {spec.name}: that head's 192 packed-projection "
+                      f"columns over {spec.t} frames plus its attention, NumPy float64, {el:.1f} s"}
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    spec = inputs.ENCODER_WORKLOADS[args.workload]
+    inp = inputs.make_encoder_inputs(spec)
+    for i in range(args.warmup):
+        oracle_sample(spec, inp, i)
+    t0 = time.perf_counter()
+    flops = 0.0
+    for i in range(args.steps):
+        flops += oracle_sample(spec, inp, i)
+    el = time.perf_counter() - t0
+    value = flops / el / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)",
+        "config": workload_config(spec),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+                         "sample": "each step: one window x one head of the workload (that head's packed-"
+                                   "projection columns and its attention), FP64 oracle on host cores"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(spec):
+    if isinstance(spec, inputs.EncoderSpec):
+        wl = (f"{spec.name}: {spec.batch} x {spec.t}-frame sequence(s), d_model {spec.d_model}, "
+              f"{spec.n_heads}x64 heads, {spec.mask.upper()} mask"
+              + (f" (chunks of {spec.chunk_len})" if spec.mask == "chunk" else ""))
+        return {"workload": wl, "batch": spec.batch, "t": spec.t, "d_model": spec.d_model,
+                "n_heads": spec.n_heads, "head_dim": 64, "mask": spec.mask,
+                "l2": "flushed between timed steps (256 MiB write)", "parallelism": "replicas (weak)"}
+    return {"workload": f"{spec.name}: {spec.t_q} query rows ({spec.beams} beams x {spec.block}) over a "
+                        f"{spec.slots}-slot token-tree cache + cross-attention to {spec.t_enc} encoder frames",
+            "t_q": spec.t_q, "slots": spec.slots, "t_enc": spec.t_enc, "n_heads": spec.n_heads,
+            "l2": "flushed between timed steps (256 MiB write)", "parallelism": "replicas (weak)"}
+
+
+# ---------------------------------------------------------------------------
+# the GPU arm
+# ---------------------------------------------------------------------------
+
+def run_gpu(args):
+    import torch
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+    step = make_step(args.workload, device)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+    nk = len(step.kernels)
+
+    for _ in range(args.warmup):
+        step.run()
+    torch.cuda.synchronize()
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(args.steps)]
+
+    def barrier():
+        if ws > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        for i in range(args.steps):
+            flush.zero_()
+            step.run(ev[i])
+        torch.cuda.synchronize()
+    barrier()
+    per_kernel = np.zeros(nk)
+    step_ms = 0.0
+    for e in ev:
+        for k in range(nk):
+            per_kernel[k] += e[k].elapsed_time(e[k + 1])
+        step_ms += e[0].elapsed_time(e[nk])
+    local_ms = step_ms / args.steps
+    per_kernel /= args.steps
+    ms = reduce_step_time(local_ms, device)
+
+    # end to end through the same calls, host buffers, copies inside the timed region
+    e2e_ms = None
+    if not args.skip_e2e:
+        for _ in range(max(1, args.warmup // 2)):
+            step.run_e2e()
+        torch.cuda.synchronize()
+        n_e2e = max(1, min(args.steps, args.e2e_steps))
+        eev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n_e2e)]
+        barrier()
+        torch.cuda.synchronize()
+        for i in range(n_e2e):
+            step.run_e2e(eev[i])
+        torch.cuda.synchronize()
+        barrier()
+        e2e_local = sum(a.elapsed_time(b) for a, b in eev) / n_e2e
+        e2e_ms = reduce_step_time(e2e_local, device)
+
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, peak_kind = load_peaks()
+    spec = step.spec
+    is_encoder = isinstance(step, EncoderStep)
+    flops = step.total_flops()
+    value = whole_job_rate(flops, ws, ms) / 1e12
+    top = int(np.argmax(per_kernel))
+    kname = step.kernels[top]
+    if is_encoder:
+        peak = peaks["bf16_tflops"]
+        achieved = step.flops[kname] / (per_kernel[top] * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": stored_traffic(kname, args.workload),
+                "kernel": kname, "peak_source": f"{peak_kind} bf16_tflops (burst); fp16 dense rate = bf16 rate",
+                "algorithmic_flops_per_launch": step.flops[kname], "launch_us": per_kernel[top] * 1e3}
+        metric, unit = METRIC, "TFLOP/s"
+    else:
+        peak = peaks["hbm_gbs"]
+        achieved = step.bytes[kname] / (per_kernel[top] * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": stored_traffic(kname, args.workload), "kernel": kname,
+                "peak_source": f"{peak_kind} hbm_gbs", "algorithmic_bytes_per_launch": step.bytes[kname],
+                "launch_us": per_kernel[top] * 1e3}
+        metric, unit = "verify+cross attention TFLOP/s (HBM-bound; see roofline)", "TFLOP/s"
+    all_kernels = {}
+    for k, name in enumerate(step.kernels):
+        ent = {"launch_us": per_kernel[k] * 1e3,
+               "tflops": step.flops[name] / (per_kernel[k] * 1e-3) / 1e12}
+        if not is_encoder:
+            ent["gbs"] = step.bytes[name] / (per_kernel[k] * 1e-3) / 1e9
+        all_kernels[name] = ent
+    cpu = None
+    if not args.skip_cpu_baseline and is_encoder:
+        cpu = time_oracle(spec, seconds=args.cpu_seconds)
+    line = {
+        "metric": metric, "value": value, "unit": unit, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic (seeded; random-init weights)",
+        "config": workload_config(spec),
+        "pct_of_peak": 100.0 * value / (peaks["bf16_tflops"] * ws),
+        "units_per_s": {k: v * ws / (ms * 1e-3) for k, v in step.units().items()},
+        "roofline": roof,
+        "kernels": all_kernels,
+        "cpu_baseline": cpu,
+        "e2e": None if e2e_ms is None else {
+            "value": whole_job_rate(flops, ws, e2e_ms) / 1e12, "unit": unit,
+            "h2d_bytes_per_step": step.h2d_bytes, "d2h_bytes_per_step": step.d2h_bytes,
+            "ms_per_step": e2e_ms},
+        "gpu_launches": step.launches_per_step * args.steps,
+        "clocks": clocks.summary(),
+        "kernel_source_hash": kernel_source_hash(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def parse(argv=None):
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["native", "reference"], default="native")
+    p.add_argument("--workload", default="windows8",
+                   choices=sorted(inputs.ENCODER_WORKLOADS) + sorted(inputs.VERIFY_WORKLOADS))
+    p.add_argument("--e2e-steps", type=int, default=200)
+    p.add_argument("--cpu-seconds", type=float, default=10.0)
+    p.add_argument("--skip-cpu-baseline", action="store_true")
+    p.add_argument("--skip-e2e", action="store_true")
+    args = p.parse_args(argv)
+    if args.warmup < 3 and args.impl == "native":
+        p.error("--warmup must be at least 3")
+    return args
+
+
+def main(argv=None):
+    argv = sys.argv[1:] if argv is None else argv
+    args = parse(argv)
+    ws, _, _ = dist_env()
+    if args.impl == "reference":
+        return run_reference(args)
+    if args.gpus > 1 and ws == 1:
+        return relaunch_under_torchrun(args.gpus, argv)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

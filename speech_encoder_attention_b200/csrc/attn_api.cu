@@ -87,9 +87,13 @@ attn_status device_info(DeviceInfo** out) {
     if (cudaGetSymbolAddress(&err, g_error_word) != cudaSuccess) return ATTN_ERR_CUDA;
     if (cudaFuncSetAttribute(sea::gemm::qkv_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              sea::gemm::SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(sea::fa::flash_attn_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(sea::fa::flash_attn_kernel<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              sea::fa::Cfg<1>::SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(sea::fa::flash_attn_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(sea::fa::flash_attn_kernel<2, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             sea::fa::Cfg<2>::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(sea::fa::flash_attn_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             sea::fa::Cfg<1>::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(sea::fa::flash_attn_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              sea::fa::Cfg<2>::SMEM_BYTES) != cudaSuccess)
       return ATTN_ERR_CUDA;
     d.num_sms = sms;
@@ -269,12 +273,13 @@ attn_status launch_attention(attn_mat q, attn_mat k, attn_mat v, int32_t batch, 
   p.limit_ns = sea::kDefaultTimeoutNs;
 
   dim3 grid(ceil_div(pl.q_tiles, pl.nq) * pl.kv_splits, n_heads, batch);
+  const bool slot = p.mask_kind == sea::fa::kSlotmask;
   if (pl.nq == 2) {
-    sea::fa::flash_attn_kernel<2>
-        <<<grid, sea::fa::Cfg<2>::THREADS, sea::fa::Cfg<2>::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    auto kern = slot ? sea::fa::flash_attn_kernel<2, true> : sea::fa::flash_attn_kernel<2, false>;
+    kern<<<grid, sea::fa::Cfg<2>::THREADS, sea::fa::Cfg<2>::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   } else {
-    sea::fa::flash_attn_kernel<1>
-        <<<grid, sea::fa::Cfg<1>::THREADS, sea::fa::Cfg<1>::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    auto kern = slot ? sea::fa::flash_attn_kernel<1, true> : sea::fa::flash_attn_kernel<1, false>;
+    kern<<<grid, sea::fa::Cfg<1>::THREADS, sea::fa::Cfg<1>::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   }
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   if (pl.kv_splits > 1) {

@@ -75,19 +75,23 @@ struct Cfg {
   static constexpr int PRODUCER_WARP = 4 * NQ;
   static constexpr int MMA_WARP = 4 * NQ + 1;
   static constexpr int TMEM_COLS = NQ == 1 ? 256 : 512;
+  // S (128 fp32 columns) of query tile q; P (fp16 pairs) overwrites its first 64.
   __host__ __device__ static constexpr uint32_t S_COL(int q) { return 128u * q; }
   __host__ __device__ static constexpr uint32_t O_COL(int q) { return 128u * NQ + 64u * q; }
-  __host__ __device__ static constexpr uint32_t P_COL(int q) { return 128u * NQ + 64u * NQ + 64u * q; }
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + NQ * TILE_BYTES;
   static constexpr int OFF_V = OFF_K + STAGES * TILE_BYTES;
   static constexpr int OFF_BARS = OFF_V + STAGES * TILE_BYTES;
-  // q_full, k_full[S], v_full[S], kv_empty[S], s_full[NQ], s_free[NQ], p_full[NQ], o_done[NQ], drain
-  static constexpr int NUM_BARS = 1 + 3 * STAGES + 4 * NQ + 1;
+  // q_full, k_full[S], v_full[S], kv_empty[S], s_full[NQ], p_full[NQ], o_done[NQ], drain
+  static constexpr int NUM_BARS = 1 + 3 * STAGES + 3 * NQ + 1;
   static constexpr int OFF_FLAGS = OFF_BARS + 8 * NUM_BARS;
   static constexpr int OFF_MISC = OFF_FLAGS + 4 * MAX_FLAG_WORDS;
   static constexpr int SMEM_BYTES = 1024 + OFF_MISC + 16;
 };
+
+// Lazy rescaling: the exponent reference m only moves when a row's max grows
+// by more than this (log2 units), so p <= 2^8 fits fp16 and O is rescaled rarely.
+constexpr float RESCALE_THRESHOLD = 8.0f;
 
 struct TileGeom {
   int q0;     // first query row (sequence-local)
@@ -108,7 +112,9 @@ __device__ __forceinline__ TileGeom q_tile_geom(const Params& p, int qt) {
   return g;
 }
 
-template <int NQ>
+// SLOT selects the bitmask family (SLOTMASK) at compile time; the range family
+// (FULL, CHUNK) carries no bitmask code in its inner loop.
+template <int NQ, bool SLOT>
 __global__ void __launch_bounds__(Cfg<NQ>::THREADS, 1)
     flash_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const Params p) {
@@ -122,10 +128,9 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, 1)
   auto v_full = [&](int s) { return bar0 + 8u * (1 + STAGES + s); };
   auto kv_empty = [&](int s) { return bar0 + 8u * (1 + 2 * STAGES + s); };
   auto s_full = [&](int q) { return bar0 + 8u * (1 + 3 * STAGES + q); };
-  auto s_free = [&](int q) { return bar0 + 8u * (1 + 3 * STAGES + NQ + q); };
-  auto p_full = [&](int q) { return bar0 + 8u * (1 + 3 * STAGES + 2 * NQ + q); };
-  auto o_done = [&](int q) { return bar0 + 8u * (1 + 3 * STAGES + 3 * NQ + q); };
-  const uint32_t drain_bar = bar0 + 8u * (1 + 3 * STAGES + 4 * NQ);
+  auto p_full = [&](int q) { return bar0 + 8u * (1 + 3 * STAGES + NQ + q); };
+  auto o_done = [&](int q) { return bar0 + 8u * (1 + 3 * STAGES + 2 * NQ + q); };
+  const uint32_t drain_bar = bar0 + 8u * (1 + 3 * STAGES + 3 * NQ);
   uint32_t* flags = reinterpret_cast<uint32_t*>(smem + C::OFF_FLAGS);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + C::OFF_MISC + 4);
@@ -163,7 +168,7 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, 1)
   const int n_kv = (kv_hi - kv_lo + BKV - 1) / BKV;
   const int j_begin = min(n_kv, split * p.kv_tiles_per_split);
   const int j_end = min(n_kv, j_begin + p.kv_tiles_per_split);
-  const bool use_flags = p.mask_kind == kSlotmask;
+  constexpr bool use_flags = SLOT;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -174,7 +179,6 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, 1)
     }
     for (int q = 0; q < NQ; ++q) {
       mbar_init(s_full(q), 1);
-      mbar_init(s_free(q), 4);
       mbar_init(p_full(q), 4);
       mbar_init(o_done(q), 1);
     }
@@ -203,7 +207,7 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, 1)
       (use_flags && row_ok) ? p.bits + static_cast<int64_t>(row_glob) * p.words_per_row : nullptr;
 
   // SLOTMASK: mark key tiles that any row of this CTA may see.
-  if (use_flags) {
+  if constexpr (use_flags) {
     if (mask_row != nullptr) {
       for (int j = j_begin; j < j_end; ++j) {
         const int w0 = j * (BKV / 32);
@@ -250,27 +254,25 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, 1)
   } else if (warp == C::MMA_WARP) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
+      // Per key tile and query tile q: O_q += P_q V (previous tile), then
+      // S_q = Q_q K^T (this tile). P_q lives in S_q's columns, so the new S
+      // must follow the PV that reads P; both are issued by this thread, and
+      // the commit after S_q tells the softmax warps that PV has finished too.
       constexpr uint32_t idesc_s = idesc_f16_f32(BQ, BKV, 0, 0);  // Q, K both K-major
       constexpr uint32_t idesc_o = idesc_f16_f32(BQ, DH, 0, 1);   // P K-major (TMEM), V MN-major
       bool ok = mbar_wait(q_full, 0, wc);
       int it = 0;
       int prev_st = 0;
-      auto issue_pv = [&](int st, int idx) -> bool {
-        if (!mbar_wait(v_full(st), (idx / STAGES) & 1, wc)) return false;
+      auto issue_pv = [&](int q, int st, int idx) -> bool {
+        if (!mbar_wait(p_full(q), idx & 1, wc)) return false;
+        tc_fence_after();
         const uint32_t sv = sbase + C::OFF_V + st * TILE_BYTES;
 #pragma unroll
-        for (int q = 0; q < NQ; ++q) {
-          if (!mbar_wait(p_full(q), idx & 1, wc)) return false;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < BKV / 16; ++kk) {
-            const uint64_t vd = smem_desc_sw128(sv + kk * 2048, TILE_BYTES, 1024);
-            mma_f16_ts(tmem_base + C::O_COL(q), tmem_base + C::P_COL(q) + kk * 8, vd, idesc_o,
-                       (idx > 0 || kk > 0) ? 1u : 0u);
-          }
-          mma_commit(o_done(q));
+        for (int kk = 0; kk < BKV / 16; ++kk) {
+          const uint64_t vd = smem_desc_sw128(sv + kk * 2048, TILE_BYTES, 1024);
+          mma_f16_ts(tmem_base + C::O_COL(q), tmem_base + C::S_COL(q) + kk * 8, vd, idesc_o,
+                     (idx > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(kv_empty(st));
         return true;
       };
       for (int j = j_begin; j < j_end && ok; ++j) {
@@ -280,10 +282,14 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, 1)
           ok = false;
           break;
         }
+        if (it > 0 && !mbar_wait(v_full(prev_st), ((it - 1) / STAGES) & 1, wc)) {
+          ok = false;
+          break;
+        }
         const uint32_t sk = sbase + C::OFF_K + st * TILE_BYTES;
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
-          if (it > 0 && !mbar_wait(s_free(q), (it - 1) & 1, wc)) {
+          if (it > 0 && !issue_pv(q, prev_st, it - 1)) {
             ok = false;
             break;
           }
@@ -298,14 +304,18 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, 1)
           mma_commit(s_full(q));
         }
         if (!ok) break;
-        if (it > 0 && !issue_pv(prev_st, it - 1)) {
-          ok = false;
-          break;
-        }
+        if (it > 0) mma_commit(kv_empty(prev_st));
         prev_st = st;
         ++it;
       }
-      if (ok && it > 0) issue_pv(prev_st, it - 1);
+      if (ok && it > 0 && mbar_wait(v_full(prev_st), ((it - 1) / STAGES) & 1, wc)) {
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) {
+          if (!issue_pv(q, prev_st, it - 1)) break;
+          mma_commit(o_done(q));
+        }
+        mma_commit(kv_empty(prev_st));
+      }
       mma_commit(drain_bar);
       mbar_wait_drain(drain_bar, 0, p.limit_ns);
     }
@@ -315,7 +325,6 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, 1)
     const uint32_t lane_field = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t s_tmem = tmem_base + C::S_COL(q) + lane_field;
     const uint32_t o_tmem = tmem_base + C::O_COL(q) + lane_field;
-    const uint32_t p_tmem = tmem_base + C::P_COL(q) + lane_field;
     // Allowed key range of this row for FULL / CHUNK (sequence-local indices).
     int lo_i = 0, hi_i = p.t_kv;
     if (p.mask_kind == kChunk) {
@@ -327,7 +336,7 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, 1)
       hi_i = 0;
     }
     const float sl2 = p.scale_log2;
-    float m_run = -INFINITY;
+    float m_run = -INFINITY;  // exponent reference (log2 units), lags the true max by < 8
     float l_run = 0.f;
     int it = 0;
     bool ok = true;
@@ -346,12 +355,9 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, 1)
 #pragma unroll
         for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(r[e]);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_free(q));
 
       const int kv0 = kv_lo + j * BKV;
-      if (use_flags) {
+      if constexpr (use_flags) {
         uint32_t wbits[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -371,48 +377,50 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, 1)
             if (e < a || e >= bnd) s[e] = -INFINITY;
         }
       }
-      float mx = s[0];
+      // row max: eight independent chains, then a short tree
+      float mx8[8];
 #pragma unroll
-      for (int e = 1; e < 128; ++e) mx = fmaxf(mx, s[e]);
-      const float m_new = fmaxf(m_run, mx * sl2);
+      for (int i = 0; i < 8; ++i) mx8[i] = s[i];
+#pragma unroll
+      for (int e = 8; e < 128; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], s[e]);
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      const float mx_l2 = mx * sl2;
+      // Move the reference only when the max grew by more than the threshold.
+      const bool grow = mx_l2 > m_run + RESCALE_THRESHOLD;
+      const float m_new = grow ? mx_l2 : m_run;
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      const float alpha = ex2_approx(m_run - m_use);
-      float sum = 0.f;
-      uint32_t pk[64];
+      const float alpha = grow ? ex2_approx(m_run - m_use) : 1.f;
+      // p = 2^(s*scale*log2e - m), summed in fp32, written as fp16 pairs over
+      // the first 64 columns of S in four chunks of 32 keys.
+      float sum8[8];
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const float p0 = ex2_approx(fmaf(s[2 * i], sl2, -m_use));
-        const float p1 = ex2_approx(fmaf(s[2 * i + 1], sl2, -m_use));
-        sum += p0 + p1;
-        pk[i] = pack_half2(p0, p1);
+      for (int i = 0; i < 8; ++i) sum8[i] = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = ex2_approx(fmaf(s[32 * c + 2 * i], sl2, -m_use));
+          const float p1 = ex2_approx(fmaf(s[32 * c + 2 * i + 1], sl2, -m_use));
+          sum8[i & 7] += p0 + p1;
+          pk[i] = pack_half2(p0, p1);
+        }
+        tmem_st16(s_tmem + c * 16, pk);
       }
+      const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
       l_run = l_run * alpha + sum;
-      if (it > 0) {
-        if (!mbar_wait(o_done(q), (it - 1) & 1, wc)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+      // O holds the PV of every earlier tile (the s_full commit covers it), and
+      // this tile's PV is only issued after p_full, so rescale it now.
+      if (it > 0 && __any_sync(0xffffffffu, grow)) {
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+          uint32_t r[32];
+          tmem_ld32(o_tmem + c * 32, r);
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            uint32_t r[32];
-            tmem_ld32(o_tmem + c * 32, r);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-            tmem_st32(o_tmem + c * 32, r);
-          }
+          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+          tmem_st32(o_tmem + c * 32, r);
         }
-      }
-      {
-        uint32_t r0[32], r1[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          r0[e] = pk[e];
-          r1[e] = pk[32 + e];
-        }
-        tmem_st32(p_tmem, r0);
-        tmem_st32(p_tmem + 32, r1);
       }
       tc_fence_before();
       __syncwarp();
@@ -422,42 +430,43 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, 1)
     }
 
     // ---------------- epilogue ----------------
-    float o[64];
-#pragma unroll
-    for (int e = 0; e < 64; ++e) o[e] = 0.f;
-    if (ok && it > 0 && mbar_wait(o_done(q), (it - 1) & 1, wc)) {
-      tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t r[32];
+    // O / l (or the unnormalised split partial), 32 columns at a time.
+    const bool have_o = ok && it > 0 && mbar_wait(o_done(q), 0, wc);
+    if (have_o) tc_fence_after();
+    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+    const int64_t part =
+        ((static_cast<int64_t>(split) * p.batch + b) * p.n_heads + h) * p.t_q + row_glob;
+#pragma unroll 1
+    for (int c = 0; c < 2; ++c) {
+      uint32_t r[32];
+      if (have_o) {
         tmem_ld32(o_tmem + c * 32, r);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) o[c * 32 + e] = __uint_as_float(r[e]);
-      }
-    }
-    if (row_ok) {
-      if (p.kv_splits > 1) {
-        const int64_t idx =
-            ((static_cast<int64_t>(split) * p.batch + b) * p.n_heads + h) * p.t_q + row_glob;
-        float4* dst = reinterpret_cast<float4*>(p.ws_o + idx * DH);
-#pragma unroll
-        for (int v = 0; v < 16; ++v) dst[v] = make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
-        reinterpret_cast<float2*>(p.ws_ml)[idx] = make_float2(m_run, l_run);
       } else {
-        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-        __half* dst = p.out + (static_cast<int64_t>(b) * p.t_q + row_glob) * p.out_stride + h * DH;
-        uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-        for (int v = 0; v < 8; ++v) {
+        for (int e = 0; e < 32; ++e) r[e] = 0u;
+      }
+      if (!row_ok) continue;
+      if (p.kv_splits > 1) {
+        float4* dst = reinterpret_cast<float4*>(p.ws_o + part * DH + c * 32);
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+          dst[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                               __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+      } else {
+        uint4* dst = reinterpret_cast<uint4*>(
+            p.out + (static_cast<int64_t>(b) * p.t_q + row_glob) * p.out_stride + h * DH + c * 32);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
           uint4 u;
-          u.x = pack_half2(o[8 * v + 0] * inv, o[8 * v + 1] * inv);
-          u.y = pack_half2(o[8 * v + 2] * inv, o[8 * v + 3] * inv);
-          u.z = pack_half2(o[8 * v + 4] * inv, o[8 * v + 5] * inv);
-          u.w = pack_half2(o[8 * v + 6] * inv, o[8 * v + 7] * inv);
-          d4[v] = u;
+          u.x = pack_half2(__uint_as_float(r[8 * v + 0]) * inv, __uint_as_float(r[8 * v + 1]) * inv);
+          u.y = pack_half2(__uint_as_float(r[8 * v + 2]) * inv, __uint_as_float(r[8 * v + 3]) * inv);
+          u.z = pack_half2(__uint_as_float(r[8 * v + 4]) * inv, __uint_as_float(r[8 * v + 5]) * inv);
+          u.w = pack_half2(__uint_as_float(r[8 * v + 6]) * inv, __uint_as_float(r[8 * v + 7]) * inv);
+          dst[v] = u;
         }
       }
     }
+    if (row_ok && p.kv_splits > 1) reinterpret_cast<float2*>(p.ws_ml)[part] = make_float2(m_run, l_run);
   }
 
   __syncwarp();
