@@ -165,13 +165,13 @@ FaPlan plan_forward(int batch, int t_q, int t_kv, int n_heads, int mask_kind, in
     pl.seg_len = chunk_len >= sea::fa::BQ ? chunk_len : (sea::fa::BQ / chunk_len) * chunk_len;
     pl.tiles_per_seg = ceil_div(pl.seg_len, sea::fa::BQ);
     pl.q_tiles = ceil_div(t_q, pl.seg_len) * pl.tiles_per_seg;
-    pl.nq = (pl.tiles_per_seg % 2 == 0) ? 2 : 1;
+    pl.nq = 1;
     pl.n_kv_max = ceil_div(pl.seg_len, sea::fa::BKV) + 1;
   } else {
     pl.seg_len = t_q;
     pl.tiles_per_seg = ceil_div(t_q, sea::fa::BQ);
     pl.q_tiles = pl.tiles_per_seg;
-    pl.nq = pl.q_tiles >= 2 ? 2 : 1;
+    pl.nq = 1;
     pl.n_kv_max = ceil_div(t_kv, sea::fa::BKV);
   }
   pl.kv_splits = 1;

@@ -40,7 +40,6 @@ namespace fa {
 constexpr int BQ = 128;
 constexpr int BKV = 128;
 constexpr int DH = 64;
-constexpr int STAGES = 3;
 constexpr int TILE_BYTES = 128 * DH * 2;  // 16 KB, one 128-row x 64-col fp16 tile
 constexpr int MAX_FLAG_WORDS = 16;        // SLOTMASK: up to 512 key tiles (65536 slots)
 
@@ -70,20 +69,29 @@ struct Params {
 
 template <int NQ>
 struct Cfg {
-  static constexpr int SOFTMAX_THREADS = 128 * NQ;
+  // One softmax warpgroup per query tile, one thread per score row.
+  static constexpr int SOFTMAX_WARPS = 4 * NQ;
+  static constexpr int SOFTMAX_THREADS = 32 * SOFTMAX_WARPS;
+  static constexpr int PRODUCER_WARP = SOFTMAX_WARPS;
+  static constexpr int MMA_WARP = SOFTMAX_WARPS + 1;
   static constexpr int THREADS = SOFTMAX_THREADS + 64;
-  static constexpr int PRODUCER_WARP = 4 * NQ;
-  static constexpr int MMA_WARP = 4 * NQ + 1;
   static constexpr int TMEM_COLS = NQ == 1 ? 256 : 512;
-  // S (128 fp32 columns) of query tile q; P (fp16 pairs) overwrites its first 64.
+  // Single-tile CTAs run two per SM (256 tensor-memory columns and a 2-stage
+  // K/V ring each), so one CTA's MMAs fill the other's pipeline drains.
+  static constexpr int STAGES = NQ == 1 ? 2 : 3;
+  static constexpr int MIN_BLOCKS = NQ == 1 ? 2 : 1;
+  // Per query tile q: S (128 fp32 columns), O (64 fp32), P (64 columns of fp16
+  // pairs). P has its own columns so the next S can be computed while the
+  // softmax of this one runs.
   __host__ __device__ static constexpr uint32_t S_COL(int q) { return 128u * q; }
   __host__ __device__ static constexpr uint32_t O_COL(int q) { return 128u * NQ + 64u * q; }
+  __host__ __device__ static constexpr uint32_t P_COL(int q) { return 128u * NQ + 64u * NQ + 64u * q; }
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + NQ * TILE_BYTES;
   static constexpr int OFF_V = OFF_K + STAGES * TILE_BYTES;
   static constexpr int OFF_BARS = OFF_V + STAGES * TILE_BYTES;
-  // q_full, k_full[S], v_full[S], kv_empty[S], s_full[NQ], p_full[NQ], o_done[NQ], drain
-  static constexpr int NUM_BARS = 1 + 3 * STAGES + 3 * NQ + 1;
+  // q_full, k_full[S], v_full[S], kv_empty[S], s_full[NQ], s_free[NQ], p_full[NQ], o_done[NQ], drain
+  static constexpr int NUM_BARS = 1 + 3 * STAGES + 4 * NQ + 1;
   static constexpr int OFF_FLAGS = OFF_BARS + 8 * NUM_BARS;
   static constexpr int OFF_MISC = OFF_FLAGS + 4 * MAX_FLAG_WORDS;
   static constexpr int SMEM_BYTES = 1024 + OFF_MISC + 16;
@@ -92,6 +100,11 @@ struct Cfg {
 // Lazy rescaling: the exponent reference m only moves when a row's max grows
 // by more than this (log2 units), so p <= 2^8 fits fp16 and O is rescaled rarely.
 constexpr float RESCALE_THRESHOLD = 8.0f;
+
+// Bit k set: pair k (mod 8) of every 16 keys takes the FMA-pipe exp2 instead
+// of MUFU ex2. Measured on B200 the extra instructions cost more than the
+// MUFU relief buys in this kernel, so no pair is moved.
+constexpr uint32_t POLY_PAIRS = 0x00u;
 
 struct TileGeom {
   int q0;     // first query row (sequence-local)
@@ -115,7 +128,7 @@ __device__ __forceinline__ TileGeom q_tile_geom(const Params& p, int qt) {
 // SLOT selects the bitmask family (SLOTMASK) at compile time; the range family
 // (FULL, CHUNK) carries no bitmask code in its inner loop.
 template <int NQ, bool SLOT>
-__global__ void __launch_bounds__(Cfg<NQ>::THREADS, 1)
+__global__ void __launch_bounds__(Cfg<NQ>::THREADS, Cfg<NQ>::MIN_BLOCKS)
     flash_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const Params p) {
   using C = Cfg<NQ>;
@@ -125,12 +138,13 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, 1)
   const uint32_t bar0 = sbase + C::OFF_BARS;
   const uint32_t q_full = bar0;
   auto k_full = [&](int s) { return bar0 + 8u * (1 + s); };
-  auto v_full = [&](int s) { return bar0 + 8u * (1 + STAGES + s); };
-  auto kv_empty = [&](int s) { return bar0 + 8u * (1 + 2 * STAGES + s); };
-  auto s_full = [&](int q) { return bar0 + 8u * (1 + 3 * STAGES + q); };
-  auto p_full = [&](int q) { return bar0 + 8u * (1 + 3 * STAGES + NQ + q); };
-  auto o_done = [&](int q) { return bar0 + 8u * (1 + 3 * STAGES + 2 * NQ + q); };
-  const uint32_t drain_bar = bar0 + 8u * (1 + 3 * STAGES + 3 * NQ);
+  auto v_full = [&](int s) { return bar0 + 8u * (1 + C::STAGES + s); };
+  auto kv_empty = [&](int s) { return bar0 + 8u * (1 + 2 * C::STAGES + s); };
+  auto s_full = [&](int q) { return bar0 + 8u * (1 + 3 * C::STAGES + q); };
+  auto s_free = [&](int q) { return bar0 + 8u * (1 + 3 * C::STAGES + NQ + q); };
+  auto p_full = [&](int q) { return bar0 + 8u * (1 + 3 * C::STAGES + 2 * NQ + q); };
+  auto o_done = [&](int q) { return bar0 + 8u * (1 + 3 * C::STAGES + 3 * NQ + q); };
+  const uint32_t drain_bar = bar0 + 8u * (1 + 3 * C::STAGES + 4 * NQ);
   uint32_t* flags = reinterpret_cast<uint32_t*>(smem + C::OFF_FLAGS);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + C::OFF_MISC + 4);
@@ -172,13 +186,14 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(k_full(s), 1);
       mbar_init(v_full(s), 1);
       mbar_init(kv_empty(s), 1);
     }
     for (int q = 0; q < NQ; ++q) {
       mbar_init(s_full(q), 1);
+      mbar_init(s_free(q), 4);
       mbar_init(p_full(q), 4);
       mbar_init(o_done(q), 1);
     }
@@ -197,12 +212,11 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, 1)
   const uint32_t tmem_base = *tmem_slot;
   const WaitCtl wc{abort_flag, p.err, p.limit_ns};
 
-  // Softmax-thread identity (meaningful for threadIdx.x < SOFTMAX_THREADS).
-  const int sq = threadIdx.x >> 7;          // query tile of this thread
-  const int srow = threadIdx.x & 127;       // row within the tile == TMEM lane
-  const int qsel = sq < NQ ? sq : 0;
-  const int row_glob = geom[qsel].q0 + srow;  // sequence-local query row
-  const bool row_ok = threadIdx.x < C::SOFTMAX_THREADS && srow < geom[qsel].rows;
+  // Softmax-thread identity (meaningful for warp < SOFTMAX_WARPS).
+  const int sq = min(warp >> 2, NQ - 1);     // query tile of this thread
+  const int srow = (warp & 3) * 32 + lane;   // row within the tile == TMEM lane
+  const int row_glob = geom[sq].q0 + srow;   // sequence-local query row
+  const bool row_ok = warp < C::SOFTMAX_WARPS && srow < geom[sq].rows;
   const uint32_t* mask_row =
       (use_flags && row_ok) ? p.bits + static_cast<int64_t>(row_glob) * p.words_per_row : nullptr;
 
@@ -234,8 +248,8 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, 1)
       int it = 0;
       for (int j = j_begin; j < j_end; ++j) {
         if (!tile_on(j)) continue;
-        const int st = it % STAGES;
-        const uint32_t ph = (it / STAGES) & 1;
+        const int st = it % C::STAGES;
+        const uint32_t ph = (it / C::STAGES) & 1;
         if (!mbar_wait(kv_empty(st), ph ^ 1u, wc)) break;
         const int kv0 = kv_lo + j * BKV;
         mbar_arrive_expect_tx(k_full(st), TILE_BYTES);
@@ -246,85 +260,85 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, 1)
       }
       // Let the copies land before the CTA may exit.
       mbar_wait_drain(q_full, 0, p.limit_ns);
-      for (int i = max(0, it - STAGES); i < it; ++i) {
-        mbar_wait_drain(k_full(i % STAGES), (i / STAGES) & 1, p.limit_ns);
-        mbar_wait_drain(v_full(i % STAGES), (i / STAGES) & 1, p.limit_ns);
+      for (int i = max(0, it - C::STAGES); i < it; ++i) {
+        mbar_wait_drain(k_full(i % C::STAGES), (i / C::STAGES) & 1, p.limit_ns);
+        mbar_wait_drain(v_full(i % C::STAGES), (i / C::STAGES) & 1, p.limit_ns);
       }
     }
   } else if (warp == C::MMA_WARP) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
-      // Per key tile and query tile q: O_q += P_q V (previous tile), then
-      // S_q = Q_q K^T (this tile). P_q lives in S_q's columns, so the new S
-      // must follow the PV that reads P; both are issued by this thread, and
-      // the commit after S_q tells the softmax warps that PV has finished too.
+      // Key tile i: S_q(i) = Q_q K(i)^T as soon as the softmax of query tile q
+      // has copied S_q(i-1) out of tensor memory, then O_q += P_q(i-1) V(i-1)
+      // once that softmax has written P_q(i-1).
       constexpr uint32_t idesc_s = idesc_f16_f32(BQ, BKV, 0, 0);  // Q, K both K-major
       constexpr uint32_t idesc_o = idesc_f16_f32(BQ, DH, 0, 1);   // P K-major (TMEM), V MN-major
+      // Descriptors are computed once; advancing K by 16 moves the start
+      // address by 32 bytes (Q, K: 2 in descriptor units) or by 16 rows of
+      // 128 bytes (V: 128 units); stages are TILE_BYTES (1024 units) apart.
+      const uint64_t q_desc0 = smem_desc_sw128(sbase + C::OFF_Q, 16, 1024);
+      const uint64_t k_desc0 = smem_desc_sw128(sbase + C::OFF_K, 16, 1024);
+      const uint64_t v_desc0 = smem_desc_sw128(sbase + C::OFF_V, TILE_BYTES, 1024);
+      constexpr uint64_t kTileUnits = TILE_BYTES >> 4;
       bool ok = mbar_wait(q_full, 0, wc);
       int it = 0;
       int prev_st = 0;
-      auto issue_pv = [&](int q, int st, int idx) -> bool {
-        if (!mbar_wait(p_full(q), idx & 1, wc)) return false;
-        tc_fence_after();
-        const uint32_t sv = sbase + C::OFF_V + st * TILE_BYTES;
+      auto issue_pv = [&](int st, int idx) -> bool {
+        if (!mbar_wait(v_full(st), (idx / C::STAGES) & 1, wc)) return false;
+        const uint64_t vd = v_desc0 + st * kTileUnits;
 #pragma unroll
-        for (int kk = 0; kk < BKV / 16; ++kk) {
-          const uint64_t vd = smem_desc_sw128(sv + kk * 2048, TILE_BYTES, 1024);
-          mma_f16_ts(tmem_base + C::O_COL(q), tmem_base + C::S_COL(q) + kk * 8, vd, idesc_o,
-                     (idx > 0 || kk > 0) ? 1u : 0u);
+        for (int q = 0; q < NQ; ++q) {
+          if (!mbar_wait(p_full(q), idx & 1, wc)) return false;
+          tc_fence_after();
+          const uint32_t o_t = tmem_base + C::O_COL(q), p_t = tmem_base + C::P_COL(q);
+#pragma unroll
+          for (int kk = 0; kk < BKV / 16; ++kk)
+            mma_f16_ts(o_t, p_t + kk * 8, vd + kk * 128, idesc_o, (idx > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(o_done(q));
         }
+        mma_commit(kv_empty(st));
         return true;
       };
       for (int j = j_begin; j < j_end && ok; ++j) {
         if (!tile_on(j)) continue;
-        const int st = it % STAGES;
-        if (!mbar_wait(k_full(st), (it / STAGES) & 1, wc)) {
+        const int st = it % C::STAGES;
+        if (!mbar_wait(k_full(st), (it / C::STAGES) & 1, wc)) {
           ok = false;
           break;
         }
-        if (it > 0 && !mbar_wait(v_full(prev_st), ((it - 1) / STAGES) & 1, wc)) {
-          ok = false;
-          break;
-        }
-        const uint32_t sk = sbase + C::OFF_K + st * TILE_BYTES;
+        const uint64_t kd = k_desc0 + st * kTileUnits;
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
-          if (it > 0 && !issue_pv(q, prev_st, it - 1)) {
+          if (it > 0 && !mbar_wait(s_free(q), (it - 1) & 1, wc)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sq_addr = sbase + C::OFF_Q + q * TILE_BYTES;
+          const uint64_t qd = q_desc0 + q * kTileUnits;
+          const uint32_t s_t = tmem_base + C::S_COL(q);
 #pragma unroll
-          for (int kk = 0; kk < DH / 16; ++kk) {
-            const uint64_t qd = smem_desc_sw128(sq_addr + kk * 32, 16, 1024);
-            const uint64_t kd = smem_desc_sw128(sk + kk * 32, 16, 1024);
-            mma_f16_ss(tmem_base + C::S_COL(q), qd, kd, idesc_s, kk > 0 ? 1u : 0u);
-          }
+          for (int kk = 0; kk < DH / 16; ++kk) mma_f16_ss(s_t, qd + kk * 2, kd + kk * 2, idesc_s, kk > 0 ? 1u : 0u);
           mma_commit(s_full(q));
         }
         if (!ok) break;
-        if (it > 0) mma_commit(kv_empty(prev_st));
+        if (it > 0 && !issue_pv(prev_st, it - 1)) {
+          ok = false;
+          break;
+        }
         prev_st = st;
         ++it;
       }
-      if (ok && it > 0 && mbar_wait(v_full(prev_st), ((it - 1) / STAGES) & 1, wc)) {
-#pragma unroll
-        for (int q = 0; q < NQ; ++q) {
-          if (!issue_pv(q, prev_st, it - 1)) break;
-          mma_commit(o_done(q));
-        }
-        mma_commit(kv_empty(prev_st));
-      }
+      if (ok && it > 0) issue_pv(prev_st, it - 1);
       mma_commit(drain_bar);
       mbar_wait_drain(drain_bar, 0, p.limit_ns);
     }
-  } else {
+  } else if (warp < C::SOFTMAX_WARPS) {
     // ---------------- softmax / correction / epilogue ----------------
     const int q = sq;
     const uint32_t lane_field = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t s_tmem = tmem_base + C::S_COL(q) + lane_field;
     const uint32_t o_tmem = tmem_base + C::O_COL(q) + lane_field;
+    const uint32_t p_tmem = tmem_base + C::P_COL(q) + lane_field;
     // Allowed key range of this row for FULL / CHUNK (sequence-local indices).
     int lo_i = 0, hi_i = p.t_kv;
     if (p.mask_kind == kChunk) {
@@ -348,15 +362,18 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, 1)
       }
       tc_fence_after();
       float s[128];
+      {
+        uint32_t r[128];
+        tmem_ld128(s_tmem, r);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(s_tmem + c * 32, r);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(r[e]);
+        for (int e = 0; e < 128; ++e) s[e] = __uint_as_float(r[e]);
       }
+      // S is in registers: the next tile's S may overwrite it.
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free(q));
 
-      const int kv0 = kv_lo + j * BKV;
+      const int kv0 = kv_lo + j * BKV;  // key index of s[0]
       if constexpr (use_flags) {
         uint32_t wbits[4];
 #pragma unroll
@@ -377,41 +394,63 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, 1)
             if (e < a || e >= bnd) s[e] = -INFINITY;
         }
       }
-      // row max: eight independent chains, then a short tree
-      float mx8[8];
+      // row max: eight independent chains of 3-input max, then a short tree
+      float mx;
+      {
+        float mx8[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mx8[i] = s[i];
+        for (int i = 0; i < 8; ++i) mx8[i] = s[i];
 #pragma unroll
-      for (int e = 8; e < 128; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], s[e]);
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        for (int e = 8; e < 128; e += 16) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mx8[i] = fmax3(mx8[i], s[e + i], s[e + 8 + i]);
+        }
+        mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
+      }
       const float mx_l2 = mx * sl2;
       // Move the reference only when the max grew by more than the threshold.
       const bool grow = mx_l2 > m_run + RESCALE_THRESHOLD;
       const float m_new = grow ? mx_l2 : m_run;
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
       const float alpha = grow ? ex2_approx(m_run - m_use) : 1.f;
-      // p = 2^(s*scale*log2e - m), summed in fp32, written as fp16 pairs over
-      // the first 64 columns of S in four chunks of 32 keys.
-      float sum8[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) sum8[i] = 0.f;
+      // P and O are still read by the previous tile's PV until it completes.
+      if (it > 0) {
+        if (!mbar_wait(o_done(q), (it - 1) & 1, wc)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+      }
+      // p = 2^(s*scale*log2e - m), summed in fp32 and written to P as fp16
+      // pairs, 32 keys at a time. MUFU ex2 serves 16 lanes per clock per SM;
+      // pairs picked by POLY_PAIRS take the FMA-pipe exp2 instead.
+      const uint64_t sl2x2 = f2_pack(sl2, sl2);
+      const uint64_t negm2 = f2_pack(-m_use, -m_use);
+      uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2_approx(fmaf(s[32 * c + 2 * i], sl2, -m_use));
-          const float p1 = ex2_approx(fmaf(s[32 * c + 2 * i + 1], sl2, -m_use));
-          sum8[i & 7] += p0 + p1;
+          float x0, x1, p0, p1;
+          f2_unpack(f2_fma(f2_pack(s[32 * c + 2 * i], s[32 * c + 2 * i + 1]), sl2x2, negm2), x0, x1);
+          if ((POLY_PAIRS >> (i & 7)) & 1) {
+            exp2_poly_x2(x0, x1, p0, p1);
+          } else {
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
+          acc2[i & 3] = f2_add(acc2[i & 3], f2_pack(p0, p1));
           pk[i] = pack_half2(p0, p1);
         }
-        tmem_st16(s_tmem + c * 16, pk);
+        tmem_st16_async(p_tmem + c * 16, pk);
       }
-      const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
-      l_run = l_run * alpha + sum;
-      // O holds the PV of every earlier tile (the s_full commit covers it), and
-      // this tile's PV is only issued after p_full, so rescale it now.
+      tmem_wait_st();
+      float sum0, sum1;
+      f2_unpack(f2_add(f2_add(acc2[0], acc2[1]), f2_add(acc2[2], acc2[3])), sum0, sum1);
+      l_run = l_run * alpha + (sum0 + sum1);
+      // O holds the PV of every earlier tile (o_done above), and this tile's
+      // PV is only issued after p_full, so rescale it now.
       if (it > 0 && __any_sync(0xffffffffu, grow)) {
 #pragma unroll 1
         for (int c = 0; c < 2; ++c) {
@@ -431,7 +470,7 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, 1)
 
     // ---------------- epilogue ----------------
     // O / l (or the unnormalised split partial), 32 columns at a time.
-    const bool have_o = ok && it > 0 && mbar_wait(o_done(q), 0, wc);
+    const bool have_o = ok && it > 0 && mbar_wait(o_done(q), (it - 1) & 1, wc);
     if (have_o) tc_fence_after();
     const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
     const int64_t part =
