@@ -131,6 +131,31 @@ attn_status attn_cross(attn_mat q, attn_mat k_enc, attn_mat v_enc, int32_t batch
                        attn_stream_t stream);
 
 /*
+ * attn_cross_static_scratch -- attn_cross for callers that cannot allocate
+ * device memory.
+ * The pages describe no such entry point; it exists for hosts that may not
+ * call cudaMalloc or hand out device buffers on the hot path: an audio or
+ * speech plugin whose host owns every device allocation through its own
+ * pool, or a real-time decode loop that must not allocate between frames.
+ * Same arguments, result and error behaviour as attn_cross, without the
+ * workspace: the split-KV partials live in a fixed 4 MiB array in the
+ * library's device memory (one per device, held until the process exits).
+ *   - The first call on a device looks up that array's address; make it
+ *     before any stream capture on that device.
+ *   - A shape whose split needs more than 4 MiB (splits x batch x n_heads x
+ *     t_q x 264 bytes; splits only happen when batch*n_heads*ceil(t_q/128)
+ *     is at most half the SM count) returns ATTN_ERR_INVALID and launches
+ *     nothing.
+ *   - Every call uses the same array. Calls whose kernels may overlap on the
+ *     GPU (different streams, or other devices' threads with this device
+ *     current) race on it: order them on one stream.
+ *   - Nothing is allocated or freed.
+ */
+attn_status attn_cross_static_scratch(attn_mat q, attn_mat k_enc, attn_mat v_enc, int32_t batch, int32_t t_q,
+                                      int32_t t_enc, int32_t n_heads, int32_t head_dim, float scale,
+                                      attn_mat out, attn_stream_t stream);
+
+/*
  * attn_workspace_size -- bytes of workspace attn_forward / attn_cross use for
  * these sizes on the current device (0 when no split is planned).
  */

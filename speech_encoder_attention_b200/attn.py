@@ -59,6 +59,9 @@ SIGNATURES = {
     "attn_cross": (ctypes.c_int, [AttnMat, AttnMat, AttnMat, ctypes.c_int32, ctypes.c_int32,
                                   ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_float,
                                   AttnMat, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "attn_cross_static_scratch": (ctypes.c_int, [AttnMat, AttnMat, AttnMat, ctypes.c_int32, ctypes.c_int32,
+                                                 ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                                 ctypes.c_float, AttnMat, ctypes.c_void_p]),
     "attn_workspace_size": (ctypes.c_size_t, [ctypes.c_int32] * 6),
     "attn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "attn_debug_error_word": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_uint32)]),

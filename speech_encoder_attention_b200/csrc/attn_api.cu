@@ -291,6 +291,36 @@ attn_status launch_attention(attn_mat q, attn_mat k, attn_mat v, int32_t batch, 
   return ATTN_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Fixed scratch for attn_cross_static_scratch (no allocation by the caller).
+// ---------------------------------------------------------------------------
+
+constexpr size_t kStaticScratchBytes = size_t(4) << 20;  // 4 MiB per device
+
+// Split-KV partials (unnormalised O, running max and sum) of
+// attn_cross_static_scratch. Every device that loads this library's device
+// code holds these 4 MiB until the process exits. In host code the name below
+// only stands in for the symbol; its device address comes from
+// cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+void* g_static_scratch_ptr[kMaxDevices] = {};
+
+// Once per device, with that device current: resolve the scratch address.
+attn_status static_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (g_static_scratch_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess || ptr == nullptr) return ATTN_ERR_CUDA;
+    g_static_scratch_ptr[dev] = ptr;
+  }
+  *out = g_static_scratch_ptr[dev];
+  return ATTN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -347,6 +377,23 @@ attn_status attn_cross(attn_mat q, attn_mat k_enc, attn_mat v_enc, int32_t batch
   full.kind = ATTN_MASK_FULL;
   return launch_attention(q, k_enc, v_enc, batch, t_q, t_enc, n_heads, head_dim, full, scale, out, workspace,
                           workspace_bytes, stream);
+}
+
+attn_status attn_cross_static_scratch(attn_mat q, attn_mat k_enc, attn_mat v_enc, int32_t batch, int32_t t_q,
+                                      int32_t t_enc, int32_t n_heads, int32_t head_dim, float scale, attn_mat out,
+                                      attn_stream_t stream) {
+  DeviceInfo* dev = nullptr;
+  if (attn_status st = device_info(&dev); st != ATTN_OK) return st;
+  void* scratch = nullptr;
+  if (attn_status st = static_scratch(&scratch); st != ATTN_OK) return st;
+  // Same launch as attn_cross with the fixed scratch as its workspace: a split
+  // that needs more than kStaticScratchBytes is rejected (ATTN_ERR_INVALID)
+  // before anything is launched. Every partial the combine step reads is
+  // written earlier in the same call, so nothing has to be cleared.
+  attn_mask full{};
+  full.kind = ATTN_MASK_FULL;
+  return launch_attention(q, k_enc, v_enc, batch, t_q, t_enc, n_heads, head_dim, full, scale, out, scratch,
+                          kStaticScratchBytes, stream);
 }
 
 size_t attn_workspace_size(int32_t batch, int32_t t_q, int32_t t_kv, int32_t n_heads, int32_t head_dim,

@@ -1,0 +1,68 @@
+"""attn_cross_static_scratch: cross-attention for callers that may not allocate
+device memory (a host that owns every device allocation through its own pool,
+or a real-time decode loop that must not allocate between frames).
+
+It runs the split-KV cross-attention with its partials in the library's fixed
+device array instead of a caller workspace. Its output must match attn_cross
+(with a caller workspace) within the parity tolerance, on two calls in a row,
+and a shape whose split needs more than the fixed 4 MiB must be refused.
+This file is named to be collected last."""
+import ctypes
+
+import numpy as np
+import pytest
+
+from speech_encoder_attention_b200 import attn, inputs
+from tests.gpu_util import assert_parity, to_dev, to_np64
+
+pytestmark = pytest.mark.gpu
+
+STATIC_SCRATCH_BYTES = 4 << 20
+
+
+def _mat(t):
+    return attn.AttnMat(ctypes.c_void_p(t.data_ptr()), t.stride(0))
+
+
+def test_static_scratch_matches_workspace_entry_point_twice():
+    import torch
+    assert torch.cuda.is_available()
+    lib = attn.load_library()
+    spec = inputs.VERIFY_WORKLOADS["verify"]
+    inp = inputs.make_verify_inputs(spec)
+    q, ke, ve = (to_dev(a) for a in (inp.q, inp.k_enc, inp.v_enc))
+    d = spec.d_model
+    # the shape splits its key range, so the scratch is really used
+    need = attn.workspace_size(1, spec.t_q, spec.t_enc, spec.n_heads, attn.MASK_FULL)
+    assert 0 < need <= STATIC_SCRATCH_BYTES
+
+    want = attn.attn_cross(q, ke, ve, 1, spec.t_q, spec.t_enc, spec.n_heads)
+    torch.cuda.synchronize()
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    for call in range(2):
+        out = torch.full((spec.t_q, d), float("nan"), dtype=torch.float16, device="cuda")
+        st = lib.attn_cross_static_scratch(_mat(q), _mat(ke), _mat(ve), 1, spec.t_q, spec.t_enc, spec.n_heads,
+                                           64, 0.125, _mat(out), stream)
+        assert st == attn.ATTN_OK, attn.status_string(st)
+        torch.cuda.synchronize()
+        assert_parity(to_np64(out), to_np64(want), what=f"static scratch call {call}")
+    assert attn.debug_error_word() == (attn.ATTN_OK, 0)
+
+
+def test_static_scratch_refuses_splits_larger_than_the_array():
+    import torch
+    lib = attn.load_library()
+    # 70 query tiles of one head: the split plan needs 2 x 8960 x 264 bytes > 4 MiB
+    t_q, t_enc, heads = 128 * 70, 300, 1
+    rng = np.random.default_rng(0)
+    q = to_dev(inputs.random_f16(rng, (t_q, 64)))
+    k = to_dev(inputs.random_f16(rng, (t_enc, 64)))
+    v = to_dev(inputs.random_f16(rng, (t_enc, 64)))
+    assert attn.workspace_size(1, t_q, t_enc, heads, attn.MASK_FULL) > STATIC_SCRATCH_BYTES
+    out = torch.zeros(t_q, 64, dtype=torch.float16, device="cuda")
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    st = lib.attn_cross_static_scratch(_mat(q), _mat(k), _mat(v), 1, t_q, t_enc, heads, 64, 0.125, _mat(out),
+                                       stream)
+    torch.cuda.synchronize()
+    assert st == attn.ATTN_ERR_INVALID
+    assert torch.count_nonzero(out) == 0, "a refused call must launch nothing"
