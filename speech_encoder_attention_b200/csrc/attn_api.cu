@@ -87,14 +87,10 @@ attn_status device_info(DeviceInfo** out) {
     if (cudaGetSymbolAddress(&err, g_error_word) != cudaSuccess) return ATTN_ERR_CUDA;
     if (cudaFuncSetAttribute(sea::gemm::qkv_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              sea::gemm::SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(sea::fa::flash_attn_kernel<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             sea::fa::Cfg<1>::SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(sea::fa::flash_attn_kernel<2, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             sea::fa::Cfg<2>::SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(sea::fa::flash_attn_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             sea::fa::Cfg<1>::SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(sea::fa::flash_attn_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             sea::fa::Cfg<2>::SMEM_BYTES) != cudaSuccess)
+        cudaFuncSetAttribute(sea::fa::flash_attn_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             sea::fa::Cfg::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(sea::fa::flash_attn_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             sea::fa::Cfg::SMEM_BYTES) != cudaSuccess)
       return ATTN_ERR_CUDA;
     d.num_sms = sms;
     d.err = static_cast<uint32_t*>(err);
@@ -146,7 +142,6 @@ bool encode_seq_3d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t t, u
 }
 
 struct FaPlan {
-  int nq;
   int seg_len, tiles_per_seg, q_tiles;
   int n_kv_max;
   int kv_splits, kv_tiles_per_split;
@@ -165,21 +160,19 @@ FaPlan plan_forward(int batch, int t_q, int t_kv, int n_heads, int mask_kind, in
     pl.seg_len = chunk_len >= sea::fa::BQ ? chunk_len : (sea::fa::BQ / chunk_len) * chunk_len;
     pl.tiles_per_seg = ceil_div(pl.seg_len, sea::fa::BQ);
     pl.q_tiles = ceil_div(t_q, pl.seg_len) * pl.tiles_per_seg;
-    pl.nq = 1;
     pl.n_kv_max = ceil_div(pl.seg_len, sea::fa::BKV) + 1;
   } else {
     pl.seg_len = t_q;
     pl.tiles_per_seg = ceil_div(t_q, sea::fa::BQ);
     pl.q_tiles = pl.tiles_per_seg;
-    pl.nq = 1;
     pl.n_kv_max = ceil_div(t_kv, sea::fa::BKV);
   }
   pl.kv_splits = 1;
   pl.kv_tiles_per_split = pl.n_kv_max;
-  const int64_t base_ctas = static_cast<int64_t>(batch) * n_heads * ceil_div(pl.q_tiles, pl.nq);
+  const int64_t base_units = static_cast<int64_t>(batch) * n_heads * pl.q_tiles;
   // CHUNK tiles already fill the GPU; the split serves short query blocks.
-  if (mask_kind != sea::fa::kChunk && base_ctas * 2 <= num_sms && pl.n_kv_max >= 2) {
-    int splits = static_cast<int>(std::min<int64_t>(pl.n_kv_max, std::max<int64_t>(1, num_sms / base_ctas)));
+  if (mask_kind != sea::fa::kChunk && base_units * 2 <= num_sms && pl.n_kv_max >= 2) {
+    int splits = static_cast<int>(std::min<int64_t>(pl.n_kv_max, std::max<int64_t>(1, num_sms / base_units)));
     const int per = ceil_div(pl.n_kv_max, splits);
     splits = ceil_div(pl.n_kv_max, per);
     if (splits > 1) {
@@ -272,14 +265,19 @@ attn_status launch_attention(attn_mat q, attn_mat k, attn_mat v, int32_t batch, 
   p.err = dev->err;
   p.limit_ns = sea::kDefaultTimeoutNs;
 
-  dim3 grid(ceil_div(pl.q_tiles, pl.nq) * pl.kv_splits, n_heads, batch);
+  const int64_t units = static_cast<int64_t>(batch) * n_heads * pl.q_tiles * pl.kv_splits;
+  if (units > INT32_MAX) return ATTN_ERR_INVALID;
+  p.units = static_cast<int>(units);
   const bool slot = p.mask_kind == sea::fa::kSlotmask;
-  if (pl.nq == 2) {
-    auto kern = slot ? sea::fa::flash_attn_kernel<2, true> : sea::fa::flash_attn_kernel<2, false>;
-    kern<<<grid, sea::fa::Cfg<2>::THREADS, sea::fa::Cfg<2>::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  if (slot) {
+    // One unit per CTA (its tile flags need a pass over every row's words).
+    sea::fa::flash_attn_kernel<true>
+        <<<p.units, sea::fa::Cfg::THREADS, sea::fa::Cfg::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   } else {
-    auto kern = slot ? sea::fa::flash_attn_kernel<1, true> : sea::fa::flash_attn_kernel<1, false>;
-    kern<<<grid, sea::fa::Cfg<1>::THREADS, sea::fa::Cfg<1>::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    // Persistent: Cfg::MIN_BLOCKS CTAs per SM walk the units.
+    const int grid = static_cast<int>(std::min<int64_t>(units, int64_t(sea::fa::Cfg::MIN_BLOCKS) * dev->num_sms));
+    sea::fa::flash_attn_kernel<false>
+        <<<grid, sea::fa::Cfg::THREADS, sea::fa::Cfg::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   }
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   if (pl.kv_splits > 1) {
