@@ -8,11 +8,13 @@ from .attention import (  # noqa: F401
     allowed_chunk,
     allowed_from_bits,
     allowed_full,
+    allowed_range,
     attention,
     attention_head,
     cross_attention,
     encoder_attention,
     packed_bias,
     qkv_projection,
+    range_attention,
     slotmask_attention,
 )

@@ -29,6 +29,23 @@ matmul serves as the library primitive for the dot products.
   mask row admits only its ancestors; block verification over KV slots indexed
   by position).
 
+* Range family with per-sequence lengths, a causal flag and a band (the
+  drafter page, "Add causal attention and attention sinks to DFlash" PR text
+  and diff: the draft block's internal attention is non-causal unless the model
+  says causal; an optional sliding window; the higgs model card: valid frames
+  must not attend to silence padding; BuzzASR discussion: a shortened
+  500-position encoder input). Readings where the pages are silent: query row i
+  of a sequence with q_len valid rows and kv_len valid keys sits at key position
+  p_i = i + (kv_len - q_len) (the query block is the last q_len positions);
+  rows i >= q_len are padding and yield 0; keys j >= kv_len are never allowed;
+  causal keeps j <= p_i; a band of window w keeps |p_i - j| < w; CHUNK keeps
+  floor(p_i / len) == floor(j / len).
+* Attention sinks (same PR: optional per-head "attn_sinks" passed to the
+  attention). Reading: a sink is one extra logit sigma_h per head, in the units
+  of the scaled scores, that joins the softmax normalisation and carries no
+  value vector: o_i = sum_j e^{s_ij} v_j / (e^{sigma_h} + sum_j e^{s_ij}).
+  sigma = -inf is no sink. A row with no allowed key yields 0.
+
 Inputs arrive as fp16 arrays and are widened to float64 exactly. Nothing is
 rounded in between; the output stays float64.
 """
@@ -78,13 +95,41 @@ def allowed_from_bits(bits: np.ndarray, t_kv: int) -> np.ndarray:
     return ((bits[:, j // 32] >> (j % 32).astype(np.uint32)) & 1).astype(bool)
 
 
+def allowed_range(t_q: int, t_kv: int, *, q_len: int | None = None, kv_len: int | None = None,
+                  chunk_len: int = 0, window: int = 0, causal: bool = False) -> np.ndarray:
+    """Allowed set of the range family for one sequence, element by element
+    from the definitions in the module docstring: valid query row (i < q_len),
+    valid key (j < kv_len), and each requested condition on the query position
+    p_i = i + (kv_len - q_len)."""
+    q_len = t_q if q_len is None else q_len
+    kv_len = t_kv if kv_len is None else kv_len
+    i = np.arange(t_q)[:, None]
+    j = np.arange(t_kv)[None, :]
+    pos = i + (kv_len - q_len)
+    a = (i < q_len) & (j < kv_len)
+    if chunk_len:
+        if chunk_len < 0:
+            raise ValueError("chunk_len must be positive")
+        a &= np.floor_divide(pos, chunk_len) == j // chunk_len
+    if causal:
+        a &= j <= pos
+    if window:
+        if window < 0:
+            raise ValueError("window must be positive")
+        a &= np.abs(pos - j) < window
+    return a
+
+
 # ----------------------------------------------------------------------------
 # attention
 # ----------------------------------------------------------------------------
 
 def attention_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, allowed: np.ndarray,
-                   scale: float, return_stats: bool = False):
-    """One head: q [t_q, dh], k/v [t_kv, dh] (float64), allowed [t_q, t_kv]."""
+                   scale: float, return_stats: bool = False, sink: float | None = None):
+    """One head: q [t_q, dh], k/v [t_kv, dh] (float64), allowed [t_q, t_kv].
+    sink: optional extra logit of the normalisation (no value vector)."""
+    if sink is not None:
+        return _attention_head_sink(q, k, v, allowed, scale, float(sink))
     s = scale * (q @ k.T)
     s_masked = np.where(allowed, s, -np.inf)
     nonempty = allowed.any(axis=1)
@@ -98,17 +143,37 @@ def attention_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, allowed: np.ndar
     return o
 
 
+def _attention_head_sink(q, k, v, allowed, scale, sink):
+    """The softmax over the allowed keys plus the sink logit, shifted by the
+    largest of them; the sink's share of the weight multiplies nothing."""
+    s = scale * (q @ k.T)
+    s_masked = np.where(allowed, s, -np.inf)
+    nonempty = allowed.any(axis=1)
+    o = np.zeros((q.shape[0], v.shape[1]), dtype=np.float64)
+    if not nonempty.any():
+        return o
+    m = np.maximum(s_masked[nonempty].max(axis=1), sink)
+    p = np.where(allowed[nonempty], np.exp(s_masked[nonempty] - m[:, None]), 0.0)
+    l = p.sum(axis=1) + np.exp(sink - m)
+    o[nonempty] = (p @ v) / l[:, None]
+    return o
+
+
 def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, n_heads: int, allowed: np.ndarray,
               scale: float = 1.0 / np.sqrt(HEAD_DIM), head_dim: int = HEAD_DIM,
-              return_stats: bool = False):
+              return_stats: bool = False, sinks: np.ndarray | None = None):
     """Multi-head attention for one sequence. q [t_q, H*dh], k/v [t_kv, H*dh];
-    head h uses columns [h*dh, (h+1)*dh) of each. Returns o [t_q, H*dh] float64."""
+    head h uses columns [h*dh, (h+1)*dh) of each. Returns o [t_q, H*dh] float64.
+    sinks: optional [H] per-head sink logits."""
     q, k, v = _f64(q), _f64(k), _f64(v)
     o = np.zeros((q.shape[0], n_heads * head_dim), dtype=np.float64)
     stats = []
+    if sinks is not None and return_stats:
+        raise ValueError("stats are not exported with sinks")
     for h in range(n_heads):
         cols = slice(h * head_dim, (h + 1) * head_dim)
-        res = attention_head(q[:, cols], k[:, cols], v[:, cols], allowed, scale, return_stats)
+        sink = None if sinks is None else float(np.asarray(sinks, dtype=np.float64)[h])
+        res = attention_head(q[:, cols], k[:, cols], v[:, cols], allowed, scale, return_stats, sink)
         if return_stats:
             o[:, cols], st = res
             stats.append(st)
@@ -146,3 +211,19 @@ def cross_attention(q, k_enc, v_enc, n_heads, scale=1.0 / np.sqrt(HEAD_DIM)):
     """Decoder queries attending to every encoder frame (t_q != t_kv allowed)."""
     return attention(q, k_enc, v_enc, n_heads, allowed_full(q.shape[0], k_enc.shape[0]), scale)
 
+
+
+def range_attention(q, k, v, batch, t_q, t_kv, n_heads, *, q_lens=None, kv_lens=None, chunk_len=0,
+                    window=0, causal=False, sinks=None, scale=1.0 / np.sqrt(HEAD_DIM)):
+    """Self- or cross-attention of ``batch`` sequences (rows [b*t_q, (b+1)*t_q)
+    of q, [b*t_kv, (b+1)*t_kv) of k and v) under the range family: per-sequence
+    valid lengths, CHUNK, band, causal, and optional per-head sinks."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    out = np.zeros((batch * t_q, n_heads * HEAD_DIM), dtype=np.float64)
+    for b in range(batch):
+        allowed = allowed_range(t_q, t_kv, q_len=None if q_lens is None else int(q_lens[b]),
+                                kv_len=None if kv_lens is None else int(kv_lens[b]),
+                                chunk_len=chunk_len, window=window, causal=causal)
+        qr, kr = slice(b * t_q, (b + 1) * t_q), slice(b * t_kv, (b + 1) * t_kv)
+        out[qr] = attention(q[qr], k[kr], v[kr], n_heads, allowed, scale, sinks=sinks)
+    return out

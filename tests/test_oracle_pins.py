@@ -343,3 +343,141 @@ def test_heads_do_not_mix():
     b = oracle.attention(q2, k2, v2, 2, oracle.allowed_full(t, t))
     np.testing.assert_array_equal(a[:, :64], b[:, :64])
     assert np.abs(a[:, 64:] - b[:, 64:]).max() > 1e-3
+
+
+# ---------------------------------------------------------------------------
+# range family: per-sequence lengths, causal, band (hand-written patterns)
+# ---------------------------------------------------------------------------
+
+def _m(rows):
+    return np.array(rows, dtype=bool)
+
+
+def test_range_masks_by_hand():
+    # causal, square: keys up to and including the row itself
+    np.testing.assert_array_equal(oracle.allowed_range(4, 4, causal=True),
+                                  _m([[1, 0, 0, 0], [1, 1, 0, 0], [1, 1, 1, 0], [1, 1, 1, 1]]))
+    # causal, 2 queries at the end of 5 keys: positions 3 and 4
+    np.testing.assert_array_equal(oracle.allowed_range(2, 5, causal=True),
+                                  _m([[1, 1, 1, 1, 0], [1, 1, 1, 1, 1]]))
+    # band of window 2: |i - j| < 2
+    np.testing.assert_array_equal(oracle.allowed_range(5, 5, window=2),
+                                  _m([[1, 1, 0, 0, 0], [1, 1, 1, 0, 0], [0, 1, 1, 1, 0],
+                                      [0, 0, 1, 1, 1], [0, 0, 0, 1, 1]]))
+    # band + causal: the row itself and the one before it
+    np.testing.assert_array_equal(oracle.allowed_range(5, 5, window=2, causal=True),
+                                  _m([[1, 0, 0, 0, 0], [1, 1, 0, 0, 0], [0, 1, 1, 0, 0],
+                                      [0, 0, 1, 1, 0], [0, 0, 0, 1, 1]]))
+    # lengths: 2 valid query rows, 3 valid keys of a 4-frame buffer
+    np.testing.assert_array_equal(oracle.allowed_range(4, 4, q_len=2, kv_len=3),
+                                  _m([[1, 1, 1, 0], [1, 1, 1, 0], [0, 0, 0, 0], [0, 0, 0, 0]]))
+    # causal with lengths: the 2 queries are positions 1 and 2 of 3 keys
+    np.testing.assert_array_equal(oracle.allowed_range(4, 4, q_len=2, kv_len=3, causal=True),
+                                  _m([[1, 1, 0, 0], [1, 1, 1, 0], [0, 0, 0, 0], [0, 0, 0, 0]]))
+    # chunks of 3 with the 2 queries at positions 4 and 5 of 6 keys: chunk 1
+    np.testing.assert_array_equal(oracle.allowed_range(2, 6, chunk_len=3),
+                                  _m([[0, 0, 0, 1, 1, 1], [0, 0, 0, 1, 1, 1]]))
+    # more queries than keys: positions -1 and 0; causal leaves row 0 empty
+    np.testing.assert_array_equal(oracle.allowed_range(2, 1, causal=True), _m([[0], [1]]))
+
+
+def test_range_special_cases_reduce_to_known_masks():
+    t = 7
+    np.testing.assert_array_equal(oracle.allowed_range(t, t), oracle.allowed_full(t, t))
+    np.testing.assert_array_equal(oracle.allowed_range(t, t, window=t), oracle.allowed_full(t, t))
+    np.testing.assert_array_equal(oracle.allowed_range(t, t, window=1), np.eye(t, dtype=bool))
+    np.testing.assert_array_equal(oracle.allowed_range(t, t, chunk_len=3), oracle.allowed_chunk(t, 3))
+    np.testing.assert_array_equal(oracle.allowed_range(t, t, causal=True, window=t),
+                                  np.tril(np.ones((t, t), bool)))
+
+
+def test_zero_queries_give_prefix_window_and_length_means():
+    rng = _rng(21)
+    t = 9
+    v = rng.standard_normal((t, 64))
+    q = np.zeros((t, 64))
+    k = rng.standard_normal((t, 64))
+    causal = oracle.range_attention(q, k, v, 1, t, t, 1, causal=True)
+    for i in range(t):
+        np.testing.assert_allclose(causal[i], v[: i + 1].mean(axis=0), rtol=1e-13, atol=1e-15)
+    band = oracle.range_attention(q, k, v, 1, t, t, 1, window=3)
+    for i in range(t):
+        np.testing.assert_allclose(band[i], v[max(0, i - 2): i + 3].mean(axis=0), rtol=1e-13, atol=1e-15)
+    lens = oracle.range_attention(q, k, v, 1, t, t, 1, q_lens=[5], kv_lens=[4])
+    for i in range(5):
+        np.testing.assert_allclose(lens[i], v[:4].mean(axis=0), rtol=1e-13, atol=1e-15)
+    np.testing.assert_array_equal(lens[5:], 0.0)
+
+
+def test_lengths_equal_the_truncated_sequences():
+    """Masking the padding must give what the shortened sequence gives alone
+    (a valid frame never attends to the padding)."""
+    rng = _rng(22)
+    t, heads, lens = 12, 2, [12, 7, 1, 0]
+    q, k, v = (rng.standard_normal((len(lens) * t, 64 * heads)) for _ in range(3))
+    got = oracle.range_attention(q, k, v, len(lens), t, t, heads, q_lens=lens, kv_lens=lens)
+    for b, n in enumerate(lens):
+        r = slice(b * t, b * t + n)
+        if n:
+            want = oracle.attention(q[r], k[r], v[r], heads, oracle.allowed_full(n, n))
+            np.testing.assert_allclose(got[r], want, rtol=1e-13, atol=1e-15)
+        np.testing.assert_array_equal(got[b * t + n:(b + 1) * t], 0.0)
+
+
+def test_range_bruteforce_causal_band_lengths():
+    rng = _rng(23)
+    t_q, t_kv, heads = 5, 8, 2
+    q = rng.standard_normal((t_q, 64 * heads))
+    k = rng.standard_normal((t_kv, 64 * heads))
+    v = rng.standard_normal((t_kv, 64 * heads))
+    # q_len 4, kv_len 7: positions 3, 4, 5, 6; causal band of 3 -> keys p-2 .. p
+    lists = [[1, 2, 3], [2, 3, 4], [3, 4, 5], [4, 5, 6], []]
+    got = oracle.range_attention(q, k, v, 1, t_q, t_kv, heads, q_lens=[4], kv_lens=[7], window=3, causal=True)
+    want = _brute_force(q.tolist(), k.tolist(), v.tolist(), lists, heads)
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-14)
+
+
+# ---------------------------------------------------------------------------
+# attention sinks
+# ---------------------------------------------------------------------------
+
+def test_sink_two_keys_closed_form():
+    s0, s1, sigma = 0.75, -1.25, 0.5
+    q = np.zeros((1, 64)); q[0, 0] = 8.0  # scale 1/8: scores equal k[:, 0]
+    k = np.zeros((2, 64)); k[0, 0], k[1, 0] = s0, s1
+    v = np.zeros((2, 64)); v[0, 1], v[1, 1] = 3.0, -2.0
+    got = oracle.attention(q, k, v, 1, oracle.allowed_full(1, 2), sinks=np.array([sigma]))
+    den = math.exp(sigma) + math.exp(s0) + math.exp(s1)
+    assert got[0, 1] == pytest.approx((3.0 * math.exp(s0) - 2.0 * math.exp(s1)) / den, rel=1e-14)
+    np.testing.assert_array_equal(np.delete(got[0], 1), 0.0)
+
+
+def test_sink_minus_inf_is_no_sink_and_zero_queries_close_form():
+    rng = _rng(24)
+    t, heads = 6, 2
+    q, k, v = (rng.standard_normal((t, 64 * heads)) for _ in range(3))
+    a = oracle.allowed_range(t, t, causal=True)
+    np.testing.assert_allclose(oracle.attention(q, k, v, heads, a, sinks=np.array([-np.inf, -np.inf])),
+                               oracle.attention(q, k, v, heads, a), rtol=1e-14, atol=1e-16)
+    sig = np.array([0.3, -2.0])
+    got = oracle.attention(np.zeros_like(q), k, v, heads, a, sinks=sig)
+    for i in range(t):
+        for h in range(heads):
+            cols = slice(64 * h, 64 * h + 64)
+            want = v[: i + 1, cols].sum(axis=0) / (math.exp(sig[h]) + i + 1)
+            np.testing.assert_allclose(got[i, cols], want, rtol=1e-13, atol=1e-15)
+
+
+def test_sink_edge_cases():
+    rng = _rng(25)
+    t = 5
+    q, k, v = (rng.standard_normal((t, 128)) for _ in range(3))
+    a = oracle.allowed_full(t, t)
+    a[2] = False
+    big = oracle.attention(q, k, v, 2, a, sinks=np.array([60.0, 0.0]))
+    assert np.abs(big[:, :64]).max() < 1e-15   # the sink takes almost all the weight
+    np.testing.assert_array_equal(big[2], 0.0)  # empty row stays zero
+    # changing head 1's sink leaves head 0 exactly as it was
+    other = oracle.attention(q, k, v, 2, a, sinks=np.array([60.0, -5.0]))
+    np.testing.assert_array_equal(big[:, :64], other[:, :64])
+    assert np.abs(big[:, 64:] - other[:, 64:]).max() > 1e-3
