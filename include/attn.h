@@ -14,7 +14,11 @@
  *     drafter's flash cross-attention.
  *   - "higgs-audio-v3-stt GGUF" model card, "Architecture note (chunked encoder)":
  *     4 s chunks encoded independently with within-chunk attention.
- *   - BuzzASR "danish" discussion #1: the Whisper encoder is fully bidirectional.
+ *   - BuzzASR "danish" discussion #1: the Whisper encoder is fully bidirectional;
+ *     a shortened 500-position encoder input (1000 mel frames).
+ *   - "Add causal attention and attention sinks to DFlash" (the drafter PR):
+ *     block-internal attention that is non-causal unless the model says causal,
+ *     an optional sliding window, and optional per-head attention sinks.
  *
  * Conventions for every entry point
  *   - All tensors are IEEE fp16 (binary16) in device memory unless stated.
@@ -57,9 +61,22 @@ typedef enum {
 typedef enum {
   ATTN_MASK_FULL = 0,     /* every key: the bidirectional encoder window */
   ATTN_MASK_CHUNK = 1,    /* keys in the query's chunk of chunk_len frames */
-  ATTN_MASK_SLOTMASK = 2  /* keys whose bit is set in the query row's bitmask */
+  ATTN_MASK_SLOTMASK = 2, /* keys whose bit is set in the query row's bitmask */
+  ATTN_MASK_BAND = 3      /* keys within `window` positions of the query (sliding window) */
 } attn_mask_kind;
 
+/*
+ * FULL, CHUNK and BAND form the range family. For sequence b with Q valid
+ * query rows and KV valid keys (q_lens[b] and kv_lens[b], or t_q and t_kv when
+ * the pointer is NULL), query row i sits at key position p_i = i + KV - Q: a
+ * query block is the last Q positions of its keys (the same row index when
+ * t_q == t_kv and no lengths are given). Row i may see key j iff
+ *   i < Q and j < KV                          (padding never attends nor is seen)
+ *   and CHUNK: floor(p_i / chunk_len) == floor(j / chunk_len)
+ *   and BAND:  |p_i - j| < window
+ *   and, if causal, j <= p_i.
+ * Rows with no visible key (including padding rows i >= Q) yield zeros.
+ */
 typedef struct {
   int32_t kind;            /* attn_mask_kind */
   int32_t chunk_len;       /* CHUNK: frames per chunk, > 0. Chunks start at frame 0
@@ -69,7 +86,14 @@ typedef struct {
                               i*words_per_row + j/32 is set (LSB first). Shared by
                               all heads and all sequences of the batch. 4-byte aligned. */
   int32_t words_per_row;   /* SLOTMASK: >= ceil(t_kv / 32) */
+  int32_t window;          /* BAND: >= 1 (values above t_q + t_kv act as t_q + t_kv);
+                              0 for every other kind */
+  int32_t causal;          /* 0 or 1; 1 also requires j <= p_i (range family only) */
   int32_t reserved;        /* must be 0 */
+  const int32_t *q_lens;   /* range family, optional: device pointer, [batch] int32,
+                              valid query rows per sequence; NULL = t_q. Values are
+                              clamped to [0, t_q] on the device. 4-byte aligned. */
+  const int32_t *kv_lens;  /* same for the keys; NULL = t_kv; clamped to [0, t_kv] */
 } attn_mask;
 
 typedef struct {
@@ -97,7 +121,9 @@ attn_status attn_qkv_pack(attn_mat x, const void *w_qkv, const void *b_q, const 
  * attn_forward -- multi-head flash attention with a mask
  *   o_i = sum_{j in A_i} softmax_j(scale * <q_i, k_j>) v_j     per head
  * A_i by mask.kind: FULL -> all t_kv keys; CHUNK -> keys of the same chunk
- * (requires t_q == t_kv); SLOTMASK -> keys whose bit is set in row i. A row
+ * (requires t_q == t_kv); BAND -> keys within the window; SLOTMASK -> keys
+ * whose bit is set in row i (window, causal, q_lens and kv_lens must be zero /
+ * NULL). The range family's lengths and causal flag are defined above. A row
  * with an empty A_i yields zeros.
  *   q   [batch*t_q,  n_heads*64] fp16   (row_stride >= n_heads*64)
  *   k,v [batch*t_kv, n_heads*64] fp16
@@ -117,6 +143,22 @@ attn_status attn_forward(attn_mat q, attn_mat k, attn_mat v, int32_t batch, int3
                          int32_t t_kv, int32_t n_heads, int32_t head_dim, attn_mask mask,
                          float scale, attn_mat out, void *workspace, size_t workspace_bytes,
                          attn_stream_t stream);
+
+/*
+ * attn_forward_sinks -- attn_forward with per-head attention sinks
+ * Source: the drafter PR (optional per-head "attn_sinks" tensor passed to the
+ * attention). Each head h has one extra logit sinks[h], in the units of the
+ * scaled scores, that joins the softmax normalisation and carries no value:
+ *   o_i = sum_{j in A_i} e^{s_ij} v_j / (e^{sinks[h]} + sum_{j in A_i} e^{s_ij}),
+ *   s_ij = scale * <q_i, k_j>.
+ * sinks: device pointer, [n_heads] fp32, 4-byte aligned; -INFINITY means no
+ * sink for that head; NULL makes the call identical to attn_forward. Every
+ * other argument is as for attn_forward (any mask kind).
+ */
+attn_status attn_forward_sinks(attn_mat q, attn_mat k, attn_mat v, int32_t batch, int32_t t_q,
+                               int32_t t_kv, int32_t n_heads, int32_t head_dim, attn_mask mask,
+                               const float *sinks, float scale, attn_mat out, void *workspace,
+                               size_t workspace_bytes, attn_stream_t stream);
 
 /*
  * attn_cross -- decoder queries attending to every encoder frame

@@ -8,6 +8,7 @@ CPU fallback.
 The function names match the C entry points:
     attn_qkv_pack(x, w_qkv, b_q, b_v, out=None)        -> qkv
     attn_forward(q, k, v, batch, t_q, t_kv, n_heads, mask=..., out=None) -> out
+    attn_forward with sinks=...                          -> attn_forward_sinks
     attn_cross(q, k_enc, v_enc, batch, t_q, t_enc, n_heads, out=None)   -> out
 """
 from __future__ import annotations
@@ -29,6 +30,7 @@ ATTN_ERR_TIMEOUT = 4
 MASK_FULL = 0
 MASK_CHUNK = 1
 MASK_SLOTMASK = 2
+MASK_BAND = 3
 
 HEAD_DIM = 64
 DEFAULT_SCALE = 0.125  # 1/sqrt(64)
@@ -44,7 +46,11 @@ class AttnMask(ctypes.Structure):
         ("chunk_len", ctypes.c_int32),
         ("bits", ctypes.c_void_p),
         ("words_per_row", ctypes.c_int32),
+        ("window", ctypes.c_int32),
+        ("causal", ctypes.c_int32),
         ("reserved", ctypes.c_int32),
+        ("q_lens", ctypes.c_void_p),
+        ("kv_lens", ctypes.c_void_p),
     ]
 
 
@@ -56,6 +62,10 @@ SIGNATURES = {
                                     ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, AttnMask,
                                     ctypes.c_float, AttnMat, ctypes.c_void_p, ctypes.c_size_t,
                                     ctypes.c_void_p]),
+    "attn_forward_sinks": (ctypes.c_int, [AttnMat, AttnMat, AttnMat, ctypes.c_int32, ctypes.c_int32,
+                                          ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, AttnMask,
+                                          ctypes.c_void_p, ctypes.c_float, AttnMat, ctypes.c_void_p,
+                                          ctypes.c_size_t, ctypes.c_void_p]),
     "attn_cross": (ctypes.c_int, [AttnMat, AttnMat, AttnMat, ctypes.c_int32, ctypes.c_int32,
                                   ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_float,
                                   AttnMat, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
@@ -149,12 +159,26 @@ def attn_qkv_pack(x, w_qkv, b_q=None, b_v=None, out=None, stream=None):
     return out
 
 
-def make_mask(kind: int = MASK_FULL, chunk_len: int = 0, bits=None) -> AttnMask:
+def _lens_ptr(t):
+    import torch
+    if t is None:
+        return 0
+    if t.dtype != torch.int32 or t.dim() != 1 or not t.is_contiguous():
+        raise ValueError("sequence lengths must be a contiguous [batch] int32 CUDA tensor")
+    return _ptr(t).value or 0
+
+
+def make_mask(kind: int = MASK_FULL, chunk_len: int = 0, bits=None, window: int = 0, causal: bool = False,
+              q_lens=None, kv_lens=None) -> AttnMask:
     import torch
     m = AttnMask()
     m.kind = kind
     m.chunk_len = chunk_len
+    m.window = window
+    m.causal = 1 if causal else 0
     m.reserved = 0
+    m.q_lens = _lens_ptr(q_lens)
+    m.kv_lens = _lens_ptr(kv_lens)
     if kind == MASK_SLOTMASK:
         if bits is None or bits.dtype not in (torch.int32, torch.uint32) or bits.dim() != 2:
             raise ValueError("SLOTMASK needs a [t_q, words_per_row] int32/uint32 CUDA tensor")
@@ -182,20 +206,30 @@ def _workspace(nbytes: int, device, workspace=None):
 
 
 def attn_forward(q, k, v, batch, t_q, t_kv, n_heads, mask_kind=MASK_FULL, chunk_len=0, bits=None,
-                 scale=DEFAULT_SCALE, out=None, workspace=None, split=True, stream=None):
+                 scale=DEFAULT_SCALE, out=None, workspace=None, split=True, stream=None, window=0,
+                 causal=False, q_lens=None, kv_lens=None, sinks=None):
     """Masked multi-head flash attention. q [batch*t_q, >=H*64] (or a column
     view of the packed qkv buffer), k/v [batch*t_kv, >=H*64]; returns out
-    [batch*t_q, H*64] fp16."""
+    [batch*t_q, H*64] fp16. window / causal / q_lens / kv_lens select the
+    range family's band, causal flag and per-sequence lengths ([batch] int32
+    CUDA tensors); sinks ([n_heads] fp32 CUDA tensor) calls attn_forward_sinks."""
     import torch
     lib = load_library()
-    mask = make_mask(mask_kind, chunk_len, bits)
+    mask = make_mask(mask_kind, chunk_len, bits, window, causal, q_lens, kv_lens)
     if out is None:
         out = torch.empty(batch * t_q, n_heads * HEAD_DIM, dtype=torch.float16, device=q.device)
     need = workspace_size(batch, t_q, t_kv, n_heads, mask_kind) if split else 0
     ws, ws_bytes = _workspace(need, q.device, workspace) if split else (None, 0)
-    st = lib.attn_forward(_mat(q), _mat(k), _mat(v), batch, t_q, t_kv, n_heads, HEAD_DIM, mask,
-                          float(scale), _mat(out), _ptr(ws), ws_bytes, _stream_ptr(stream))
-    _check(st, "attn_forward")
+    if sinks is None:
+        st = lib.attn_forward(_mat(q), _mat(k), _mat(v), batch, t_q, t_kv, n_heads, HEAD_DIM, mask,
+                              float(scale), _mat(out), _ptr(ws), ws_bytes, _stream_ptr(stream))
+        _check(st, "attn_forward")
+        return out
+    if sinks.dtype != torch.float32 or sinks.dim() != 1 or not sinks.is_contiguous():
+        raise ValueError("sinks must be a contiguous [n_heads] float32 CUDA tensor")
+    st = lib.attn_forward_sinks(_mat(q), _mat(k), _mat(v), batch, t_q, t_kv, n_heads, HEAD_DIM, mask,
+                                _ptr(sinks), float(scale), _mat(out), _ptr(ws), ws_bytes, _stream_ptr(stream))
+    _check(st, "attn_forward_sinks")
     return out
 
 

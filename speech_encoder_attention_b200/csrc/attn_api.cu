@@ -87,9 +87,13 @@ attn_status device_info(DeviceInfo** out) {
     if (cudaGetSymbolAddress(&err, g_error_word) != cudaSuccess) return ATTN_ERR_CUDA;
     if (cudaFuncSetAttribute(sea::gemm::qkv_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              sea::gemm::SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(sea::fa::flash_attn_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(sea::fa::flash_attn_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              sea::fa::Cfg::SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(sea::fa::flash_attn_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(sea::fa::flash_attn_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             sea::fa::Cfg::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(sea::fa::flash_attn_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             sea::fa::Cfg::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(sea::fa::flash_attn_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              sea::fa::Cfg::SMEM_BYTES) != cudaSuccess)
       return ATTN_ERR_CUDA;
     d.num_sms = sms;
@@ -190,8 +194,8 @@ bool valid_mat(const attn_mat& m, int64_t cols) {
 }
 
 attn_status launch_attention(attn_mat q, attn_mat k, attn_mat v, int32_t batch, int32_t t_q, int32_t t_kv,
-                             int32_t n_heads, int32_t head_dim, attn_mask mask, float scale, attn_mat out,
-                             void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+                             int32_t n_heads, int32_t head_dim, attn_mask mask, const float* sinks, float scale,
+                             attn_mat out, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   // ---- validation (host only, before any CUDA call) ----
   if (batch <= 0 || t_q <= 0 || t_kv <= 0 || n_heads <= 0) return ATTN_ERR_INVALID;
   if (head_dim != sea::fa::DH) return ATTN_ERR_INVALID;
@@ -202,13 +206,21 @@ attn_status launch_attention(attn_mat q, attn_mat k, attn_mat v, int32_t batch, 
   const int64_t cols = static_cast<int64_t>(n_heads) * head_dim;
   if (!valid_mat(q, cols) || !valid_mat(k, cols) || !valid_mat(v, cols) || !valid_mat(out, cols))
     return ATTN_ERR_INVALID;
+  auto misaligned4 = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 3u) != 0; };
   if (mask.reserved != 0) return ATTN_ERR_INVALID;
+  if (mask.causal != 0 && mask.causal != 1) return ATTN_ERR_INVALID;
+  if (mask.kind != ATTN_MASK_BAND && mask.window != 0) return ATTN_ERR_INVALID;
+  if (misaligned4(mask.q_lens) || misaligned4(mask.kv_lens) || misaligned4(sinks)) return ATTN_ERR_INVALID;
   if (mask.kind == ATTN_MASK_CHUNK) {
     if (mask.chunk_len <= 0 || t_q != t_kv) return ATTN_ERR_INVALID;
   } else if (mask.kind == ATTN_MASK_SLOTMASK) {
-    if (mask.bits == nullptr || (reinterpret_cast<uintptr_t>(mask.bits) & 3u) != 0) return ATTN_ERR_INVALID;
+    if (mask.bits == nullptr || misaligned4(mask.bits)) return ATTN_ERR_INVALID;
     if (t_kv > sea::fa::MAX_FLAG_WORDS * 32 * sea::fa::BKV) return ATTN_ERR_INVALID;
     if (mask.words_per_row < (t_kv + 31) / 32) return ATTN_ERR_INVALID;
+    // the bits define the allowed set alone
+    if (mask.causal != 0 || mask.q_lens != nullptr || mask.kv_lens != nullptr) return ATTN_ERR_INVALID;
+  } else if (mask.kind == ATTN_MASK_BAND) {
+    if (mask.window <= 0) return ATTN_ERR_INVALID;
   } else if (mask.kind != ATTN_MASK_FULL) {
     return ATTN_ERR_INVALID;
   }
@@ -251,6 +263,14 @@ attn_status launch_attention(attn_mat q, attn_mat k, attn_mat v, int32_t batch, 
   if (mask.kind == ATTN_MASK_CHUNK && mask.chunk_len >= t_q) p.mask_kind = sea::fa::kFull;
   p.bits = mask.kind == ATTN_MASK_SLOTMASK ? mask.bits : nullptr;
   p.words_per_row = mask.kind == ATTN_MASK_SLOTMASK ? mask.words_per_row : 0;
+  // |p_i - j| never exceeds t_q + t_kv, so a wider window changes nothing.
+  p.window = mask.kind == ATTN_MASK_BAND
+                 ? static_cast<int>(std::min<int64_t>(mask.window, static_cast<int64_t>(t_q) + t_kv + 1))
+                 : 0;
+  p.causal = mask.causal;
+  p.q_lens = mask.q_lens;
+  p.kv_lens = mask.kv_lens;
+  p.sinks = sinks;
   p.seg_len = pl.seg_len;
   p.tiles_per_seg = pl.tiles_per_seg;
   p.q_tiles = pl.q_tiles;
@@ -269,21 +289,30 @@ attn_status launch_attention(attn_mat q, attn_mat k, attn_mat v, int32_t batch, 
   if (units > INT32_MAX) return ATTN_ERR_INVALID;
   p.units = static_cast<int>(units);
   const bool slot = p.mask_kind == sea::fa::kSlotmask;
+  // The lengths / causal / BAND / sinks code is compiled into its own variant.
+  const bool ext = p.mask_kind == sea::fa::kBand || p.causal != 0 || p.q_lens != nullptr ||
+                   p.kv_lens != nullptr || p.sinks != nullptr;
+  const int threads = sea::fa::Cfg::THREADS;
+  const int smem = sea::fa::Cfg::SMEM_BYTES;
   if (slot) {
     // One unit per CTA (its tile flags need a pass over every row's words).
-    sea::fa::flash_attn_kernel<true>
-        <<<p.units, sea::fa::Cfg::THREADS, sea::fa::Cfg::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    if (ext)
+      sea::fa::flash_attn_kernel<true, true><<<p.units, threads, smem, stream>>>(tq, tk, tv, p);
+    else
+      sea::fa::flash_attn_kernel<true, false><<<p.units, threads, smem, stream>>>(tq, tk, tv, p);
   } else {
     // Persistent: Cfg::MIN_BLOCKS CTAs per SM walk the units.
     const int grid = static_cast<int>(std::min<int64_t>(units, int64_t(sea::fa::Cfg::MIN_BLOCKS) * dev->num_sms));
-    sea::fa::flash_attn_kernel<false>
-        <<<grid, sea::fa::Cfg::THREADS, sea::fa::Cfg::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    if (ext)
+      sea::fa::flash_attn_kernel<false, true><<<grid, threads, smem, stream>>>(tq, tk, tv, p);
+    else
+      sea::fa::flash_attn_kernel<false, false><<<grid, threads, smem, stream>>>(tq, tk, tv, p);
   }
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   if (pl.kv_splits > 1) {
     const int64_t rows = static_cast<int64_t>(batch) * n_heads * t_q;
     sea::fa::combine_kernel<<<ceil_div(rows, 8), 256, 0, stream>>>(
-        p.ws_o, p.ws_ml, pl.kv_splits, batch, n_heads, t_q, p.out, p.out_stride);
+        p.ws_o, p.ws_ml, pl.kv_splits, batch, n_heads, t_q, sinks, p.out, p.out_stride);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   }
   return ATTN_OK;
@@ -364,7 +393,14 @@ attn_status attn_qkv_pack(attn_mat x, const void* w_qkv, const void* b_q, const 
 attn_status attn_forward(attn_mat q, attn_mat k, attn_mat v, int32_t batch, int32_t t_q, int32_t t_kv,
                          int32_t n_heads, int32_t head_dim, attn_mask mask, float scale, attn_mat out,
                          void* workspace, size_t workspace_bytes, attn_stream_t stream) {
-  return launch_attention(q, k, v, batch, t_q, t_kv, n_heads, head_dim, mask, scale, out, workspace,
+  return launch_attention(q, k, v, batch, t_q, t_kv, n_heads, head_dim, mask, nullptr, scale, out, workspace,
+                          workspace_bytes, stream);
+}
+
+attn_status attn_forward_sinks(attn_mat q, attn_mat k, attn_mat v, int32_t batch, int32_t t_q, int32_t t_kv,
+                               int32_t n_heads, int32_t head_dim, attn_mask mask, const float* sinks, float scale,
+                               attn_mat out, void* workspace, size_t workspace_bytes, attn_stream_t stream) {
+  return launch_attention(q, k, v, batch, t_q, t_kv, n_heads, head_dim, mask, sinks, scale, out, workspace,
                           workspace_bytes, stream);
 }
 
@@ -373,8 +409,8 @@ attn_status attn_cross(attn_mat q, attn_mat k_enc, attn_mat v_enc, int32_t batch
                        size_t workspace_bytes, attn_stream_t stream) {
   attn_mask full{};
   full.kind = ATTN_MASK_FULL;
-  return launch_attention(q, k_enc, v_enc, batch, t_q, t_enc, n_heads, head_dim, full, scale, out, workspace,
-                          workspace_bytes, stream);
+  return launch_attention(q, k_enc, v_enc, batch, t_q, t_enc, n_heads, head_dim, full, nullptr, scale, out,
+                          workspace, workspace_bytes, stream);
 }
 
 attn_status attn_cross_static_scratch(attn_mat q, attn_mat k_enc, attn_mat v_enc, int32_t batch, int32_t t_q,
@@ -390,8 +426,8 @@ attn_status attn_cross_static_scratch(attn_mat q, attn_mat k_enc, attn_mat v_enc
   // written earlier in the same call, so nothing has to be cleared.
   attn_mask full{};
   full.kind = ATTN_MASK_FULL;
-  return launch_attention(q, k_enc, v_enc, batch, t_q, t_enc, n_heads, head_dim, full, scale, out, scratch,
-                          kStaticScratchBytes, stream);
+  return launch_attention(q, k_enc, v_enc, batch, t_q, t_enc, n_heads, head_dim, full, nullptr, scale, out,
+                          scratch, kStaticScratchBytes, stream);
 }
 
 size_t attn_workspace_size(int32_t batch, int32_t t_q, int32_t t_kv, int32_t n_heads, int32_t head_dim,

@@ -46,7 +46,7 @@ constexpr int DH = 64;
 constexpr int TILE_BYTES = 128 * DH * 2;  // 16 KB, one 128-row x 64-col fp16 tile
 constexpr int MAX_FLAG_WORDS = 16;        // SLOTMASK: up to 512 key tiles (65536 slots)
 
-enum MaskKind : int { kFull = 0, kChunk = 1, kSlotmask = 2 };
+enum MaskKind : int { kFull = 0, kChunk = 1, kSlotmask = 2, kBand = 3 };
 
 struct Params {
   int batch, t_q, t_kv, n_heads;
@@ -55,6 +55,12 @@ struct Params {
   int chunk_len;
   const uint32_t* bits;
   int words_per_row;
+  // range family: band window, causal flag, optional per-sequence lengths
+  int window;
+  int causal;
+  const int* q_lens;
+  const int* kv_lens;
+  const float* sinks;  // optional [n_heads] sink logits (units of the scaled scores)
   // query-tile schedule: the query axis is cut into segments of seg_len rows
   // (whole chunks for CHUNK, the whole sequence otherwise), each segment into
   // tiles_per_seg tiles of up to 128 rows.
@@ -99,6 +105,7 @@ struct Cfg {
 // Lazy rescaling: the exponent reference m only moves when a row's max grows
 // by more than this (log2 units), so p <= 2^8 fits fp16 and O is rescaled rarely.
 constexpr float RESCALE_THRESHOLD = 8.0f;
+constexpr float kLog2e = 1.4426950408889634f;
 
 // Bit k set: pair k (mod 8) of every 16 keys takes the FMA-pipe exp2 instead
 // of MUFU ex2. Measured on B200 the extra instructions cost more than the
@@ -124,6 +131,56 @@ __device__ __forceinline__ TileGeom q_tile_geom(const Params& p, int qt) {
   return g;
 }
 
+// Valid query rows and keys of one sequence, and the key position of its query
+// row 0 (a query block is the last q positions of its keys).
+struct SeqLen {
+  int q, kv, off;
+};
+
+// EXT: the launch uses lengths, causal, BAND or sinks (a separate compile-time
+// variant, so the plain FULL / CHUNK kernel carries none of that code).
+template <bool EXT>
+__device__ __forceinline__ SeqLen seq_len(const Params& p, int b) {
+  SeqLen L{p.t_q, p.t_kv, 0};
+  if constexpr (!EXT) return L;
+  if (p.q_lens != nullptr) L.q = min(max(__ldg(p.q_lens + b), 0), p.t_q);
+  if (p.kv_lens != nullptr) L.kv = min(max(__ldg(p.kv_lens + b), 0), p.t_kv);
+  L.off = L.kv - L.q;
+  return L;
+}
+
+// Keys [lo, hi) that query row i (sequence-local) of the range family may see;
+// hi <= lo means none. Both ends are non-decreasing in i.
+template <bool EXT>
+__device__ __forceinline__ void row_keys(const Params& p, const SeqLen& L, int i, int& lo, int& hi) {
+  lo = 0;
+  hi = L.kv;
+  if constexpr (!EXT) {
+    if (p.mask_kind == kChunk) {
+      lo = (i / p.chunk_len) * p.chunk_len;
+      hi = min(hi, lo + p.chunk_len);
+    }
+    return;
+  }
+  if (i >= L.q) {
+    hi = 0;
+    return;
+  }
+  const int pos = i + L.off;
+  if (p.mask_kind == kChunk) {
+    if (pos < 0) {
+      hi = 0;
+      return;
+    }
+    lo = (pos / p.chunk_len) * p.chunk_len;
+    hi = min(hi, lo + p.chunk_len);
+  } else if (p.mask_kind == kBand) {
+    lo = max(0, pos - p.window + 1);
+    hi = min(hi, pos + p.window);
+  }
+  if (p.causal) hi = min(hi, pos + 1);
+}
+
 // One work unit: a query tile of one (sequence, head) and its key-tile range.
 struct Unit {
   int b, h, split;
@@ -132,6 +189,7 @@ struct Unit {
   int j_begin, j_end;    // key tiles [j_begin, j_end) of this unit
 };
 
+template <bool EXT>
 __device__ __forceinline__ Unit decode_unit(const Params& p, int u) {
   Unit U;
   U.split = u % p.kv_splits;
@@ -143,23 +201,39 @@ __device__ __forceinline__ Unit decode_unit(const Params& p, int u) {
   const TileGeom g = q_tile_geom(p, qt);
   U.q0 = g.q0;
   U.rows = g.rows;
-  int lo = 0, hi = p.t_kv;
-  if (p.mask_kind == kChunk && g.rows > 0) {
-    lo = (g.q0 / p.chunk_len) * p.chunk_len;
-    hi = min(((g.q0 + g.rows - 1) / p.chunk_len + 1) * p.chunk_len, p.t_kv);
+  // Keys any valid row of the tile may see: the union of the rows' ranges,
+  // which (both ends being monotone) runs from the first row's start to the
+  // last valid row's end.
+  int lo = 0, hi = 0;
+  if (p.mask_kind == kSlotmask) {
+    hi = p.t_kv;
+  } else if (g.rows > 0) {
+    const SeqLen L = seq_len<EXT>(p, U.b);
+    const int last = min(g.q0 + g.rows, L.q) - 1;
+    if (last >= g.q0) {
+      int lo2, hi1;
+      row_keys<EXT>(p, L, g.q0, lo, hi1);
+      row_keys<EXT>(p, L, last, lo2, hi);
+    }
   }
+  hi = max(hi, lo);
   U.kv_lo = lo;
   const int n_kv = (hi - lo + BKV - 1) / BKV;
-  U.j_begin = min(n_kv, U.split * p.kv_tiles_per_split);
-  U.j_end = min(n_kv, U.j_begin + p.kv_tiles_per_split);
+  if (p.kv_splits == 1) {
+    U.j_begin = 0;
+    U.j_end = n_kv;
+  } else {
+    U.j_begin = min(n_kv, U.split * p.kv_tiles_per_split);
+    U.j_end = min(n_kv, U.j_begin + p.kv_tiles_per_split);
+  }
   return U;
 }
 
 // SLOT selects the bitmask family (SLOTMASK) at compile time; the range family
-// (FULL, CHUNK) carries no bitmask code and runs persistent CTAs. SLOTMASK
+// (FULL, CHUNK, BAND, with lengths and causal) carries no bitmask code and runs persistent CTAs. SLOTMASK
 // CTAs each own one unit (gridDim.x == units): the tile flags need one pass of
 // every row's mask words before any role starts.
-template <bool SLOT>
+template <bool SLOT, bool EXT>
 __global__ void __launch_bounds__(Cfg::THREADS, Cfg::MIN_BLOCKS)
     flash_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const Params p) {
@@ -221,7 +295,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, Cfg::MIN_BLOCKS)
 
   // SLOTMASK: mark the key tiles any row of this CTA's (single) unit may see.
   if constexpr (use_flags) {
-    const Unit U = decode_unit(p, blockIdx.x);
+    const Unit U = decode_unit<EXT>(p, blockIdx.x);
     if (warp < C::SOFTMAX_WARPS && srow < U.rows) {
       const uint32_t* mrow = p.bits + static_cast<int64_t>(U.q0 + srow) * p.words_per_row;
       for (int j = U.j_begin; j < U.j_end; ++j) {
@@ -246,7 +320,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, Cfg::MIN_BLOCKS)
       int qn = 0, it = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
-        const Unit U = decode_unit(p, u);
+        const Unit U = decode_unit<EXT>(p, u);
         if (U.rows == 0) continue;
         const int qb = qn & 1;
         if (!mbar_wait(q_empty(qb), ((qn >> 1) & 1) ^ 1u, wc)) break;
@@ -310,7 +384,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, Cfg::MIN_BLOCKS)
         return true;
       };
       for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
-        const Unit U = decode_unit(p, u);
+        const Unit U = decode_unit<EXT>(p, u);
         if (U.rows == 0) continue;
         const int qb = qn & 1;
         if (!mbar_wait(q_full(qb), (qn >> 1) & 1, wc)) break;
@@ -365,22 +439,15 @@ __global__ void __launch_bounds__(Cfg::THREADS, Cfg::MIN_BLOCKS)
     int it = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
-      const Unit U = decode_unit(p, u);
+      const Unit U = decode_unit<EXT>(p, u);
       if (U.rows == 0) continue;
       const int row_glob = U.q0 + srow;  // sequence-local query row
       const bool row_ok = srow < U.rows;
       const uint32_t* mask_row =
           (use_flags && row_ok) ? p.bits + static_cast<int64_t>(row_glob) * p.words_per_row : nullptr;
-      // Allowed key range of this row for FULL / CHUNK (sequence-local indices).
-      int lo_i = 0, hi_i = p.t_kv;
-      if (p.mask_kind == kChunk) {
-        lo_i = (row_glob / p.chunk_len) * p.chunk_len;
-        hi_i = min(lo_i + p.chunk_len, p.t_kv);
-      }
-      if (!row_ok) {
-        lo_i = 0;
-        hi_i = 0;
-      }
+      // Allowed key range of this row for the range family (sequence-local indices).
+      int lo_i = 0, hi_i = 0;
+      if (!use_flags && row_ok) row_keys<EXT>(p, seq_len<EXT>(p, U.b), row_glob, lo_i, hi_i);
       float m_run = -INFINITY;  // exponent reference (log2 units), lags the true max by < 8
       float l_run = 0.f;
       int t_unit = 0;  // tiles of this unit done
@@ -507,7 +574,13 @@ __global__ void __launch_bounds__(Cfg::THREADS, Cfg::MIN_BLOCKS)
       const bool have_o = t_unit > 0 && mbar_wait(o_done, (it - 1) & 1, wc);
       if (t_unit > 0 && !have_o) ok = false;
       if (have_o) tc_fence_after();
-      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      // A sink adds 2^(sink*log2e - m) to the normaliser (split partials get it
+      // in the combine step). No visible key: m = -inf, so the output is 0.
+      float l_fin = l_run;
+      if constexpr (EXT) {
+        if (p.sinks != nullptr && p.kv_splits == 1) l_fin += ex2_approx(__ldg(p.sinks + U.h) * kLog2e - m_run);
+      }
+      const float inv = l_fin > 0.f ? 1.f / l_fin : 0.f;
       const int64_t part =
           ((static_cast<int64_t>(U.split) * p.batch + U.b) * p.n_heads + U.h) * p.t_q + row_glob;
 #pragma unroll 1
@@ -560,10 +633,12 @@ __global__ void __launch_bounds__(Cfg::THREADS, Cfg::MIN_BLOCKS)
 
 
 // Merges the split-KV partials of one (sequence, head, row) per warp:
-//   M = max_s m_s,  L = sum_s l_s 2^(m_s - M),  o = sum_s O_s 2^(m_s - M) / L.
+//   M = max_s m_s,  L = sum_s l_s 2^(m_s - M) [+ 2^(sink*log2e - M)],
+//   o = sum_s O_s 2^(m_s - M) / L.
 __global__ void __launch_bounds__(256)
     combine_kernel(const float* __restrict__ ws_o, const float* __restrict__ ws_ml, int splits,
-                   int batch, int n_heads, int t_q, __half* __restrict__ out, int64_t out_stride) {
+                   int batch, int n_heads, int t_q, const float* __restrict__ sinks, __half* __restrict__ out,
+                   int64_t out_stride) {
   const int64_t rows = static_cast<int64_t>(batch) * n_heads * t_q;
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (idx >= rows) return;
@@ -588,6 +663,7 @@ __global__ void __launch_bounds__(256)
       o0 += ov.x * w;
       o1 += ov.y * w;
     }
+    if (sinks != nullptr) l += ex2_approx(__ldg(sinks + h) * kLog2e - mmax);
   }
   const float inv = l > 0.f ? 1.f / l : 0.f;
   __half2* dst = reinterpret_cast<__half2*>(out + (static_cast<int64_t>(b) * t_q + r) * out_stride + h * DH);

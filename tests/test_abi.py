@@ -94,6 +94,35 @@ def test_forward_rejects_bad_masks(lib):
     assert call_forward(lib, mask=mk) == attn.ATTN_ERR_INVALID
 
 
+def test_forward_rejects_bad_range_options(lib):
+    def mk(kind=attn.MASK_FULL, **kw):
+        x = attn.AttnMask(); x.kind = kind
+        for key, val in kw.items():
+            setattr(x, key, val)
+        return x
+    assert call_forward(lib, mask=mk(window=4)) == attn.ATTN_ERR_INVALID                # window on FULL
+    assert call_forward(lib, mask=mk(attn.MASK_BAND)) == attn.ATTN_ERR_INVALID           # BAND needs window
+    assert call_forward(lib, mask=mk(attn.MASK_BAND, window=-3)) == attn.ATTN_ERR_INVALID
+    assert call_forward(lib, mask=mk(causal=2)) == attn.ATTN_ERR_INVALID
+    assert call_forward(lib, mask=mk(q_lens=P4 + 0x1000002)) == attn.ATTN_ERR_INVALID    # misaligned
+    assert call_forward(lib, mask=mk(kv_lens=P4 + 0x1000001)) == attn.ATTN_ERR_INVALID
+    slot = dict(bits=P4 + 0x1000000, words_per_row=2)
+    assert call_forward(lib, mask=mk(attn.MASK_SLOTMASK, causal=1, **slot)) == attn.ATTN_ERR_INVALID
+    assert call_forward(lib, mask=mk(attn.MASK_SLOTMASK, kv_lens=P4 + 0x2000000, **slot)) == attn.ATTN_ERR_INVALID
+    assert call_forward(lib, mask=mk(attn.MASK_CHUNK, chunk_len=16, window=8)) == attn.ATTN_ERR_INVALID
+
+
+def test_forward_sinks_validates_like_forward(lib):
+    args = [m(P, 128), m(P2, 128), m(P3, 128), 1, 64, 64, 2, 64, full(), ctypes.c_void_p(P4 + 0x1000000),
+            0.125, m(P4, 128), ctypes.c_void_p(0), 0, None]
+    bad = list(args); bad[9] = ctypes.c_void_p(P4 + 0x1000002)   # misaligned sinks
+    assert lib.attn_forward_sinks(*bad) == attn.ATTN_ERR_INVALID
+    bad = list(args); bad[3] = 0
+    assert lib.attn_forward_sinks(*bad) == attn.ATTN_ERR_INVALID
+    bad = list(args); bad[11] = m(P + 64, 128)                     # output overlaps q
+    assert lib.attn_forward_sinks(*bad) == attn.ATTN_ERR_INVALID
+
+
 def test_cross_rejects_invalid_arguments(lib):
     args = [m(P, 128), m(P2, 128), m(P3, 128), 1, 80, 1500, 2, 64, 0.125, m(P4, 128),
             ctypes.c_void_p(0), 0, None]
