@@ -62,11 +62,27 @@ def attn_pair_flops(pairs: int, heads: int, dh: int = 64) -> float:
     return 4.0 * dh * heads * pairs
 
 
+def band_pairs(t: int, w: int) -> int:
+    """Allowed (query, key) pairs of one t-frame sequence under |i - j| < w."""
+    i = np.arange(t)
+    return int((np.minimum(t, i + w) - np.maximum(0, i - w + 1)).sum())
+
+
 def encoder_pairs(spec: inputs.EncoderSpec) -> int:
     if spec.mask == "chunk":
         full, rest = divmod(spec.t, spec.chunk_len)
         return spec.batch * (full * spec.chunk_len ** 2 + rest ** 2)
+    if spec.mask == "band":
+        return spec.batch * band_pairs(spec.t, spec.band)
+    lens = inputs.encoder_lengths(spec)
+    if lens is not None:
+        return int((lens.astype(np.int64) ** 2).sum())
     return spec.batch * spec.t * spec.t
+
+
+def encoder_valid_rows(spec: inputs.EncoderSpec) -> int:
+    lens = inputs.encoder_lengths(spec)
+    return int(lens.sum()) if lens is not None else spec.batch * spec.t
 
 
 def kernel_source_hash() -> str:
@@ -220,11 +236,14 @@ class EncoderStep:
         self.d = d
         self.qkv = torch.empty(rows, 3 * d, dtype=torch.float16, device=device)
         self.out = torch.empty(rows, d, dtype=torch.float16, device=device)
-        self.mask = attn.MASK_CHUNK if spec.mask == "chunk" else attn.MASK_FULL
+        self.mask = {"chunk": attn.MASK_CHUNK, "band": attn.MASK_BAND}.get(spec.mask, attn.MASK_FULL)
+        lens = inputs.encoder_lengths(spec)
+        self.lens = None if lens is None else dev(lens)
         self.host_x = torch.from_numpy(inp.x).pin_memory()
         self.host_out = torch.empty(rows, d, dtype=torch.float16).pin_memory()
         self.kernels = ["qkv_gemm", "flash_attn"]
-        self.flops = {"qkv_gemm": qkv_flops(rows, d),
+        # algorithmic work: the projection of the valid frames, attention over allowed pairs
+        self.flops = {"qkv_gemm": qkv_flops(encoder_valid_rows(spec), d),
                       "flash_attn": attn_pair_flops(encoder_pairs(spec), spec.n_heads)}
         self.launches_per_step = 2
 
@@ -236,7 +255,8 @@ class EncoderStep:
         if events:
             events[1].record()
         a.attn_forward(self.qkv[:, :d], self.qkv[:, d:2 * d], self.qkv[:, 2 * d:], s.batch, s.t, s.t, s.n_heads,
-                       mask_kind=self.mask, chunk_len=s.chunk_len, out=self.out, split=False)
+                       mask_kind=self.mask, chunk_len=s.chunk_len, window=s.band, q_lens=self.lens,
+                       kv_lens=self.lens, out=self.out, split=False)
         if events:
             events[2].record()
 
@@ -336,9 +356,73 @@ class VerifyStep:
         return {"query_rows": self.spec.t_q}
 
 
+class DrafterStep:
+    """The drafter's block attention: each beam's 16 queries at the end of its
+    448 keys, bidirectional or causal inside the block, with per-head sinks."""
+
+    def __init__(self, spec: inputs.DrafterSpec, device):
+        import torch
+        from speech_encoder_attention_b200 import attn
+        self.attn = attn
+        self.spec = spec
+        inp = inputs.make_drafter_inputs(spec)
+        dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+        self.q, self.k, self.v, self.sinks = dev(inp.q), dev(inp.k), dev(inp.v), dev(inp.sinks)
+        d = spec.d_model
+        self.out = torch.empty(spec.beams * spec.t_q, d, dtype=torch.float16, device=device)
+        ws = attn.workspace_size(spec.beams, spec.t_q, spec.t_kv, spec.n_heads, attn.MASK_FULL)
+        self.ws = torch.empty(max(ws, 16), dtype=torch.uint8, device=device)
+        self.split_launches = 2 if ws > 0 else 1
+        self.host_q = torch.from_numpy(inp.q).pin_memory()
+        self.host_out = torch.empty(spec.beams * spec.t_q, d, dtype=torch.float16).pin_memory()
+        per_beam = (spec.t_q * spec.context + spec.t_q * (spec.t_q + 1) // 2) if spec.causal \
+            else spec.t_q * spec.t_kv
+        self.kernels = ["drafter_attn"]
+        self.flops = {"drafter_attn": attn_pair_flops(spec.beams * per_beam, spec.n_heads)}
+        self.bytes = {"drafter_attn": 2 * d * spec.beams * (2 * spec.t_q + 2 * spec.t_kv) + 4 * spec.n_heads}
+        self.launches_per_step = self.split_launches
+
+    def run(self, events=None):
+        a, s = self.attn, self.spec
+        if events:
+            events[0].record()
+        a.attn_forward(self.q, self.k, self.v, s.beams, s.t_q, s.t_kv, s.n_heads, causal=s.causal,
+                       sinks=self.sinks, out=self.out, workspace=self.ws)
+        if events:
+            events[1].record()
+
+    def run_e2e(self, events=None):
+        if events:
+            events[0].record()
+        self.q.copy_(self.host_q, non_blocking=True)
+        self.run()
+        self.host_out.copy_(self.out, non_blocking=True)
+        if events:
+            events[-1].record()
+
+    @property
+    def h2d_bytes(self):
+        return self.host_q.numel() * 2
+
+    @property
+    def d2h_bytes(self):
+        return self.host_out.numel() * 2
+
+    def total_flops(self):
+        return sum(self.flops.values())
+
+    def total_bytes(self):
+        return sum(self.bytes.values())
+
+    def units(self):
+        return {"query_rows": self.spec.beams * self.spec.t_q}
+
+
 def make_step(name, device):
     if name in inputs.ENCODER_WORKLOADS:
         return EncoderStep(inputs.ENCODER_WORKLOADS[name], device)
+    if name in inputs.DRAFTER_WORKLOADS:
+        return DrafterStep(inputs.DRAFTER_WORKLOADS[name], device)
     return VerifyStep(inputs.VERIFY_WORKLOADS[name], device)
 
 
@@ -354,12 +438,16 @@ def oracle_sample(spec: inputs.EncoderSpec, inp, i: int):
     d, t = spec.d_model, spec.t
     b, h = i % spec.batch, i % spec.n_heads
     cols = np.r_[h * 64:(h + 1) * 64, d + h * 64:d + (h + 1) * 64, 2 * d + h * 64:2 * d + (h + 1) * 64]
-    x = inp.x[b * t:(b + 1) * t]
+    lens = inputs.encoder_lengths(spec)
+    n = t if lens is None else int(lens[b])  # valid frames of the window
+    x = inp.x[b * t:b * t + n]
     qkv = oracle.qkv_projection(x, inp.w_qkv[cols], inp.b_q[h * 64:(h + 1) * 64], inp.b_v[h * 64:(h + 1) * 64])
-    allowed = oracle.allowed_full(t, t) if spec.mask == "full" else oracle.allowed_chunk(t, spec.chunk_len)
+    if spec.mask == "chunk":
+        allowed = oracle.allowed_chunk(n, spec.chunk_len)
+    else:
+        allowed = oracle.allowed_range(n, n, window=spec.band)
     oracle.attention(qkv[:, :64], qkv[:, 64:128], qkv[:, 128:], 1, allowed)
-    pairs = encoder_pairs(inputs.EncoderSpec("s", 1, t, d, 1, spec.mask, spec.chunk_len, 0))
-    return 2.0 * t * d * 192 + attn_pair_flops(pairs, 1)
+    return 2.0 * n * d * 192 + attn_pair_flops(int(allowed.sum()), 1)
 
 
 def oracle_threads() -> int:
@@ -385,29 +473,91 @@ def time_oracle(spec, seconds: float = 10.0, max_samples: int = 400):
                       f"columns over {spec.t} frames plus its attention, NumPy float64, {el:.1f} s"}
 
 
+def workload_spec(name):
+    for table in (inputs.ENCODER_WORKLOADS, inputs.VERIFY_WORKLOADS, inputs.DRAFTER_WORKLOADS):
+        if name in table:
+            return table[name]
+    raise KeyError(name)
+
+
+def workload_metric(spec) -> str:
+    if isinstance(spec, inputs.EncoderSpec):
+        return METRIC
+    if isinstance(spec, inputs.DrafterSpec):
+        return "drafter block attention TFLOP/s (HBM-bound; see roofline)"
+    return "verify+cross attention TFLOP/s (HBM-bound; see roofline)"
+
+
+class SmallOracleStep:
+    """The whole verify or drafter step in FP64 (small enough to run entire)."""
+
+    def __init__(self, spec):
+        self.spec = spec
+        if isinstance(spec, inputs.DrafterSpec):
+            self.inp = inputs.make_drafter_inputs(spec)
+        else:
+            self.inp = inputs.make_verify_inputs(spec)
+
+    def __call__(self, i=0) -> float:
+        import oracle
+        s, inp = self.spec, self.inp
+        if isinstance(s, inputs.DrafterSpec):
+            oracle.range_attention(inp.q, inp.k, inp.v, s.beams, s.t_q, s.t_kv, s.n_heads, causal=s.causal,
+                                   sinks=inp.sinks)
+            a = oracle.allowed_range(s.t_q, s.t_kv, causal=s.causal)
+            return attn_pair_flops(s.beams * int(a.sum()), s.n_heads)
+        oracle.slotmask_attention(inp.q, inp.k_cache, inp.v_cache, inp.bits, s.n_heads)
+        oracle.cross_attention(inp.q, inp.k_enc, inp.v_enc, s.n_heads)
+        pairs = int(inputs.unpack_bits(inp.bits, s.slots).sum()) + s.t_q * s.t_enc
+        return attn_pair_flops(pairs, s.n_heads)
+
+    def describe(self, n, el):
+        return (f"{n} runs of the whole {self.spec.name} step (every row and head), NumPy float64, {el:.1f} s")
+
+
+def time_small_oracle(spec, seconds: float = 10.0, max_runs: int = 200):
+    run = SmallOracleStep(spec)
+    run()
+    t0 = time.perf_counter()
+    flops, n = 0.0, 0
+    while n < max_runs and (time.perf_counter() - t0 < seconds or n == 0):
+        flops += run(n)
+        n += 1
+    el = time.perf_counter() - t0
+    return {"value": flops / el / 1e12, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+            "sample": run.describe(n, el)}
+
+
 def run_reference(args):
     ws, rank, _ = dist_env()
     if rank != 0:
         return 0
-    spec = inputs.ENCODER_WORKLOADS[args.workload]
-    inp = inputs.make_encoder_inputs(spec)
+    spec = workload_spec(args.workload)
+    if isinstance(spec, inputs.EncoderSpec):
+        inp = inputs.make_encoder_inputs(spec)
+        sample = lambda i: oracle_sample(spec, inp, i)
+        what = ("each step: one window x one head of the workload (that head's packed-projection columns "
+                "and its attention), FP64 oracle on host cores")
+    else:
+        sample = SmallOracleStep(spec)
+        what = "each step: the whole workload (every row and head), FP64 oracle on host cores"
     for i in range(args.warmup):
-        oracle_sample(spec, inp, i)
+        sample(i)
     t0 = time.perf_counter()
     flops = 0.0
     for i in range(args.steps):
-        flops += oracle_sample(spec, inp, i)
+        flops += sample(i)
     el = time.perf_counter() - t0
     value = flops / el / 1e12
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "impl": "reference", "metric": workload_metric(spec), "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded)",
         "config": workload_config(spec),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
-                         "sample": "each step: one window x one head of the workload (that head's packed-"
-                                   "projection columns and its attention), FP64 oracle on host cores"},
+                         "sample": what},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -416,12 +566,27 @@ def run_reference(args):
 
 def workload_config(spec):
     if isinstance(spec, inputs.EncoderSpec):
+        lens = inputs.encoder_lengths(spec)
         wl = (f"{spec.name}: {spec.batch} x {spec.t}-frame sequence(s), d_model {spec.d_model}, "
               f"{spec.n_heads}x64 heads, {spec.mask.upper()} mask"
-              + (f" (chunks of {spec.chunk_len})" if spec.mask == "chunk" else ""))
-        return {"workload": wl, "batch": spec.batch, "t": spec.t, "d_model": spec.d_model,
-                "n_heads": spec.n_heads, "head_dim": 64, "mask": spec.mask,
-                "l2": "flushed between timed steps (256 MiB write)", "parallelism": "replicas (weak)"}
+              + (f" (chunks of {spec.chunk_len})" if spec.mask == "chunk" else "")
+              + (f" (window {spec.band})" if spec.mask == "band" else "")
+              + (f", valid lengths {lens.tolist()}" if lens is not None else ""))
+        cfg = {"workload": wl, "batch": spec.batch, "t": spec.t, "d_model": spec.d_model,
+               "n_heads": spec.n_heads, "head_dim": 64, "mask": spec.mask,
+               "l2": "flushed between timed steps (256 MiB write)", "parallelism": "replicas (weak)"}
+        if lens is not None:
+            cfg["valid_lengths"] = lens.tolist()
+        if spec.mask == "band":
+            cfg["window"] = spec.band
+        return cfg
+    if isinstance(spec, inputs.DrafterSpec):
+        return {"workload": f"{spec.name}: {spec.beams} beams x {spec.t_q} queries at the end of {spec.t_kv} keys, "
+                            f"{'causal' if spec.causal else 'bidirectional'} block, per-head sinks, "
+                            f"{spec.n_heads}x64 heads",
+                "beams": spec.beams, "t_q": spec.t_q, "t_kv": spec.t_kv, "causal": spec.causal,
+                "n_heads": spec.n_heads, "l2": "flushed between timed steps (256 MiB write)",
+                "parallelism": "replicas (weak)"}
     return {"workload": f"{spec.name}: {spec.t_q} query rows ({spec.beams} beams x {spec.block}) over a "
                         f"{spec.slots}-slot token-tree cache + cross-attention to {spec.t_enc} encoder frames",
             "t_q": spec.t_q, "slots": spec.slots, "t_enc": spec.t_enc, "n_heads": spec.n_heads,
@@ -431,6 +596,14 @@ def workload_config(spec):
 # ---------------------------------------------------------------------------
 # the GPU arm
 # ---------------------------------------------------------------------------
+
+def check_device_errors(step, where):
+    """A kernel whose bounded wait expired gave up (its output is void) and
+    recorded it in the library's device error word: such a run measures nothing."""
+    st, word = step.attn.debug_error_word()
+    if st != step.attn.ATTN_OK or word != 0:
+        raise RuntimeError(f"device error word {word:#x} after the {where}: a kernel wait timed out")
+
 
 def run_gpu(args):
     import torch
@@ -466,6 +639,7 @@ def run_gpu(args):
             step.run(ev[i])
         torch.cuda.synchronize()
     barrier()
+    check_device_errors(step, "timed steps")
     per_kernel = np.zeros(nk)
     step_ms = 0.0
     for e in ev:
@@ -490,6 +664,7 @@ def run_gpu(args):
             step.run_e2e(eev[i])
         torch.cuda.synchronize()
         barrier()
+        check_device_errors(step, "end-to-end steps")
         e2e_local = sum(a.elapsed_time(b) for a, b in eev) / n_e2e
         e2e_ms = reduce_step_time(e2e_local, device)
 
@@ -513,7 +688,7 @@ def run_gpu(args):
                 "frac": achieved / peak, "traffic": stored_traffic(kname, args.workload),
                 "kernel": kname, "peak_source": f"{peak_kind} bf16_tflops (burst); fp16 dense rate = bf16 rate",
                 "algorithmic_flops_per_launch": step.flops[kname], "launch_us": per_kernel[top] * 1e3}
-        metric, unit = METRIC, "TFLOP/s"
+        unit = "TFLOP/s"
     else:
         peak = peaks["hbm_gbs"]
         achieved = step.bytes[kname] / (per_kernel[top] * 1e-3) / 1e9
@@ -521,7 +696,8 @@ def run_gpu(args):
                 "traffic": stored_traffic(kname, args.workload), "kernel": kname,
                 "peak_source": f"{peak_kind} hbm_gbs", "algorithmic_bytes_per_launch": step.bytes[kname],
                 "launch_us": per_kernel[top] * 1e3}
-        metric, unit = "verify+cross attention TFLOP/s (HBM-bound; see roofline)", "TFLOP/s"
+        unit = "TFLOP/s"
+    metric = workload_metric(spec)
     all_kernels = {}
     for k, name in enumerate(step.kernels):
         ent = {"launch_us": per_kernel[k] * 1e3,
@@ -530,8 +706,9 @@ def run_gpu(args):
             ent["gbs"] = step.bytes[name] / (per_kernel[k] * 1e-3) / 1e9
         all_kernels[name] = ent
     cpu = None
-    if not args.skip_cpu_baseline and is_encoder:
-        cpu = time_oracle(spec, seconds=args.cpu_seconds)
+    if not args.skip_cpu_baseline:
+        cpu = (time_oracle(spec, seconds=args.cpu_seconds) if is_encoder
+               else time_small_oracle(spec, seconds=args.cpu_seconds))
     line = {
         "metric": metric, "value": value, "unit": unit, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -561,7 +738,8 @@ def parse(argv=None):
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", choices=["native", "reference"], default="native")
     p.add_argument("--workload", default="windows8",
-                   choices=sorted(inputs.ENCODER_WORKLOADS) + sorted(inputs.VERIFY_WORKLOADS))
+                   choices=sorted(inputs.ENCODER_WORKLOADS) + sorted(inputs.VERIFY_WORKLOADS)
+                   + sorted(inputs.DRAFTER_WORKLOADS))
     p.add_argument("--e2e-steps", type=int, default=200)
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--skip-cpu-baseline", action="store_true")

@@ -321,7 +321,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, Cfg::MIN_BLOCKS)
       bool ok = true;
       for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
         const Unit U = decode_unit<EXT>(p, u);
-        if (U.rows == 0) continue;
+        if (U.rows == 0 || (!SLOT && U.j_end <= U.j_begin)) continue;  // see the softmax's empty-unit note
         const int qb = qn & 1;
         if (!mbar_wait(q_empty(qb), ((qn >> 1) & 1) ^ 1u, wc)) break;
         mbar_arrive_expect_tx(q_full(qb), TILE_BYTES);
@@ -385,7 +385,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, Cfg::MIN_BLOCKS)
       };
       for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
         const Unit U = decode_unit<EXT>(p, u);
-        if (U.rows == 0) continue;
+        if (U.rows == 0 || (!SLOT && U.j_end <= U.j_begin)) continue;  // see the softmax's empty-unit note
         const int qb = qn & 1;
         if (!mbar_wait(q_full(qb), (qn >> 1) & 1, wc)) break;
         ++qn;  // qn now counts this unit
@@ -443,6 +443,30 @@ __global__ void __launch_bounds__(Cfg::THREADS, Cfg::MIN_BLOCKS)
       if (U.rows == 0) continue;
       const int row_glob = U.q0 + srow;  // sequence-local query row
       const bool row_ok = srow < U.rows;
+      if (!SLOT && U.j_end <= U.j_begin) {
+        // No key tile (padding rows, rows before the first key, a split past
+        // the unit's keys): the rows see no key. In the persistent kernel such
+        // a unit touches neither tensor memory nor a barrier in any role, so
+        // the softmax cannot complete barrier phases ahead of the MMA thread's
+        // parity waits. (A SLOTMASK CTA owns one unit: its empty unit takes
+        // the general path.)
+        if (row_ok) {
+          const int64_t part =
+              ((static_cast<int64_t>(U.split) * p.batch + U.b) * p.n_heads + U.h) * p.t_q + row_glob;
+          if (p.kv_splits > 1) {
+            float4* dst = reinterpret_cast<float4*>(p.ws_o + part * DH);
+#pragma unroll
+            for (int v = 0; v < DH / 4; ++v) dst[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+            reinterpret_cast<float2*>(p.ws_ml)[part] = make_float2(-INFINITY, 0.f);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<int64_t>(U.b) * p.t_q + row_glob) * p.out_stride +
+                                                  U.h * DH);
+#pragma unroll
+            for (int v = 0; v < DH / 8; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+        continue;
+      }
       const uint32_t* mask_row =
           (use_flags && row_ok) ? p.bits + static_cast<int64_t>(row_glob) * p.words_per_row : nullptr;
       // Allowed key range of this row for the range family (sequence-local indices).

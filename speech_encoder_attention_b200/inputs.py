@@ -18,6 +18,21 @@ Workloads (sizes follow the pages' encoder and decoder):
                    (11 x 200 + 125 = 2325 frames), chunk-local mask (seed 4). The
                    4 s chunk rule is the higgs-audio-v3-stt model card's
                    "Architecture note (chunked encoder)"; 4 s at 50 frames/s = 200.
+* ``varlen8``   -- 8 windows of up to 1500 frames with per-window valid lengths
+                   drawn uniformly from [500, 1500] (seed 6; lengths from the
+                   generator stream [6, 1]): the shortened 500-position input
+                   (1000 mel frames; BuzzASR discussion) up to a full window. The
+                   frames past a window's length are padding that no valid frame
+                   may attend to (higgs model card: attending to the silence
+                   padding corrupts the conditioning).
+* ``band8``     -- 8 full windows under a sliding-window band of 256 frames
+                   (seed 7). The drafter PR adds a sliding window without a size;
+                   256 frames (~5 s) is this recipe's choice.
+* ``drafter`` / ``drafter_causal`` -- the drafter's block attention: 5 beams,
+                   each a block of 16 queries (anchor + 15 drafts) at the end of
+                   448 keys (432 context positions + the block), 20 heads of 64,
+                   per-head sink logits ~ N(0, 1) (seeds 8, 9). Non-causal inside
+                   the block by default, causal when the model says so (drafter PR).
 * ``verify``    -- decoder block verification over a token tree: 5 beams x
                    (anchor + 15 drafts) = 80 query rows over a 448-slot KV cache,
                    each row limited to its ancestors, plus cross-attention of the
@@ -50,6 +65,8 @@ class EncoderSpec:
     chunk_len: int
     seed: int
     window_offset: bool = False
+    band: int = 0          # BAND window in frames (mask == "band")
+    varlen: bool = False   # per-window valid lengths, see encoder_lengths
 
 
 ENCODER_WORKLOADS: Dict[str, EncoderSpec] = {
@@ -57,7 +74,63 @@ ENCODER_WORKLOADS: Dict[str, EncoderSpec] = {
     "window": EncoderSpec("window", 1, 1500, 1280, 20, "full", 0, 2),
     "windows8": EncoderSpec("windows8", 8, 1500, 1280, 20, "full", 0, 3, True),
     "chunks": EncoderSpec("chunks", 1, 2325, 1280, 20, "chunk", 200, 4),
+    "varlen8": EncoderSpec("varlen8", 8, 1500, 1280, 20, "full", 0, 6, True, varlen=True),
+    "band8": EncoderSpec("band8", 8, 1500, 1280, 20, "band", 0, 7, True, band=256),
 }
+
+
+def encoder_lengths(spec: EncoderSpec) -> Optional[np.ndarray]:
+    """Valid frames of each window (int32 [batch]) of a varlen workload, else None:
+    uniform integers in [500, t] from the generator stream [seed, 1]."""
+    if not spec.varlen:
+        return None
+    rng = np.random.default_rng([spec.seed, 1])
+    return rng.integers(500, spec.t + 1, size=spec.batch).astype(np.int32)
+
+
+@dataclasses.dataclass(frozen=True)
+class DrafterSpec:
+    name: str
+    n_heads: int
+    d_model: int
+    block: int     # queries per beam: anchor + drafts, at the end of the keys
+    beams: int     # independent sequences
+    context: int   # key positions before the block
+    causal: bool   # block-internal attention causal (else bidirectional)
+    seed: int
+
+    @property
+    def t_q(self) -> int:
+        return self.block
+
+    @property
+    def t_kv(self) -> int:
+        return self.context + self.block
+
+
+DRAFTER_WORKLOADS: Dict[str, DrafterSpec] = {
+    "drafter": DrafterSpec("drafter", 20, 1280, 16, 5, 432, False, 8),
+    "drafter_causal": DrafterSpec("drafter_causal", 20, 1280, 16, 5, 432, True, 9),
+}
+
+
+@dataclasses.dataclass
+class DrafterInputs:
+    spec: DrafterSpec
+    q: np.ndarray      # [beams * block, d_model] float16
+    k: np.ndarray      # [beams * (context + block), d_model] float16
+    v: np.ndarray      # [beams * (context + block), d_model] float16
+    sinks: np.ndarray  # [n_heads] float32 sink logits
+
+
+def make_drafter_inputs(spec: DrafterSpec) -> DrafterInputs:
+    rng = np.random.default_rng(spec.seed)
+    d = spec.d_model
+    q = _normal_f16(rng, (spec.beams * spec.t_q, d))
+    k = _normal_f16(rng, (spec.beams * spec.t_kv, d))
+    v = _normal_f16(rng, (spec.beams * spec.t_kv, d))
+    sinks = rng.standard_normal(spec.n_heads).astype(np.float32)
+    return DrafterInputs(spec, q, k, v, sinks)
 
 
 @dataclasses.dataclass(frozen=True)

@@ -235,3 +235,81 @@ def test_sinks_with_slotmask_verify_workload():
     allowed = oracle.allowed_from_bits(inp.bits, spec.slots)
     ref = oracle.attention(inp.q, inp.k_cache, inp.v_cache, spec.n_heads, allowed, sinks=sinks)
     assert_parity(to_np64(got), ref, what="slotmask + sinks")
+
+
+# ---------------------------------------------------------------------------
+# the benchmarked workloads of these options, at full size, in the bench's
+# launch configuration
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", ["varlen8", "band8"])
+def test_encoder_workload_full_size(name):
+    torch = torch_mod()
+    spec = inputs.ENCODER_WORKLOADS[name]
+    inp = inputs.make_encoder_inputs(spec)
+    lens = inputs.encoder_lengths(spec)
+    d = spec.d_model
+    x, w, bq, bv = (to_dev(a) for a in (inp.x, inp.w_qkv, inp.b_q, inp.b_v))
+    qkv = attn.attn_qkv_pack(x, w, bq, bv)
+    dl = None if lens is None else i32(lens)
+    kind = attn.MASK_BAND if spec.mask == "band" else attn.MASK_FULL
+    out = attn.attn_forward(qkv[:, :d], qkv[:, d:2 * d], qkv[:, 2 * d:], spec.batch, spec.t, spec.t, spec.n_heads,
+                            mask_kind=kind, window=spec.band, q_lens=dl, kv_lens=dl, split=False)
+    torch.cuda.synchronize()
+    ref_qkv = oracle.qkv_projection(inp.x, inp.w_qkv, inp.b_q, inp.b_v)
+    ref = oracle.range_attention(ref_qkv[:, :d], ref_qkv[:, d:2 * d], ref_qkv[:, 2 * d:], spec.batch, spec.t, spec.t,
+                                 spec.n_heads, q_lens=lens, kv_lens=lens, window=spec.band)
+    got = to_np64(out)
+    assert_parity(to_np64(qkv), ref_qkv, what=f"{name} qkv")
+    assert_parity(got, ref, what=f"{name} attention")
+    for b in range(spec.batch):
+        n = spec.t if lens is None else int(lens[b])
+        assert_parity(got[b * spec.t:b * spec.t + n], ref[b * spec.t:b * spec.t + n], what=f"{name} window {b}")
+        np.testing.assert_array_equal(got[b * spec.t + n:(b + 1) * spec.t], 0.0)
+    st, word = attn.debug_error_word()
+    assert st == attn.ATTN_OK and word == 0
+
+
+@pytest.mark.parametrize("name", ["drafter", "drafter_causal"])
+def test_drafter_workload(name):
+    torch = torch_mod()
+    spec = inputs.DRAFTER_WORKLOADS[name]
+    inp = inputs.make_drafter_inputs(spec)
+    ws = attn.workspace_size(spec.beams, spec.t_q, spec.t_kv, spec.n_heads, attn.MASK_FULL)
+    workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device="cuda")
+    out = attn.attn_forward(to_dev(inp.q), to_dev(inp.k), to_dev(inp.v), spec.beams, spec.t_q, spec.t_kv,
+                            spec.n_heads, causal=spec.causal, sinks=f32(inp.sinks), workspace=workspace)
+    torch.cuda.synchronize()
+    ref = oracle.range_attention(inp.q, inp.k, inp.v, spec.beams, spec.t_q, spec.t_kv, spec.n_heads,
+                                 causal=spec.causal, sinks=inp.sinks)
+    assert_parity(to_np64(out), ref, what=name)
+    st, word = attn.debug_error_word()
+    assert st == attn.ATTN_OK and word == 0
+
+
+def test_many_units_without_keys_back_to_back():
+    """Units whose rows see no key (all padding) are skipped by every role; a
+    CTA that meets several in a row must not get a barrier phase ahead. Many
+    calls over a batch full of empty and one-row sequences, then the device
+    error word must still be clear."""
+    torch = torch_mod()
+    t, heads = 1500, 20
+    lens = [0, 1, 0, 130, 0, 0, 1500, 574, 0, 1, 129, 0, 0, 0, 256, 0]
+    rng = np.random.default_rng(19)
+    q, k, v = rand_qkv(rng, len(lens), t, t, heads)
+    dq, dk, dv, dl = to_dev(q), to_dev(k), to_dev(v), i32(lens)
+    for _ in range(300):
+        out = attn.attn_forward(dq, dk, dv, len(lens), t, t, heads, q_lens=dl, kv_lens=dl, split=False)
+    torch.cuda.synchronize()
+    st, word = attn.debug_error_word()
+    assert st == attn.ATTN_OK and word == 0, f"device error word {word:#x}"
+    got = to_np64(out)
+    sel = [0, 1, 3, 6, 10]
+    qs = np.concatenate([q[b * t:(b + 1) * t] for b in sel])
+    ks = np.concatenate([k[b * t:(b + 1) * t] for b in sel])
+    vs = np.concatenate([v[b * t:(b + 1) * t] for b in sel])
+    ref = oracle.range_attention(qs, ks, vs, len(sel), t, t, heads, q_lens=[lens[b] for b in sel],
+                                 kv_lens=[lens[b] for b in sel])
+    assert_parity(np.concatenate([got[b * t:(b + 1) * t] for b in sel]), ref, what="empty-unit stress")
+    for b, n in enumerate(lens):
+        np.testing.assert_array_equal(got[b * t + n:(b + 1) * t], 0.0)

@@ -83,3 +83,36 @@ def test_pack_unpack_roundtrip():
     assert bits.shape == (7, 3)
     # bits past the last slot stay clear
     assert np.all(bits[:, 2] >> np.uint32(6) == 0)
+
+
+def test_varlen_lengths_are_seeded_and_in_range():
+    spec = inputs.ENCODER_WORKLOADS["varlen8"]
+    a, b = inputs.encoder_lengths(spec), inputs.encoder_lengths(spec)
+    np.testing.assert_array_equal(a, b)
+    assert a.dtype == np.int32 and a.shape == (spec.batch,)
+    assert a.min() >= 500 and a.max() <= spec.t
+    assert inputs.encoder_lengths(inputs.ENCODER_WORKLOADS["windows8"]) is None
+
+
+def test_drafter_inputs_shapes_and_determinism():
+    spec = inputs.DRAFTER_WORKLOADS["drafter_causal"]
+    a, b = inputs.make_drafter_inputs(spec), inputs.make_drafter_inputs(spec)
+    assert a.q.shape == (spec.beams * spec.t_q, spec.d_model)
+    assert a.k.shape == a.v.shape == (spec.beams * spec.t_kv, spec.d_model)
+    assert a.sinks.shape == (spec.n_heads,) and a.sinks.dtype == np.float32
+    np.testing.assert_array_equal(a.k, b.k)
+    assert spec.t_kv == spec.context + spec.block
+
+
+def test_bench_pair_counts_match_brute_force():
+    """The bench's algorithmic flop counts: allowed pairs counted in closed form
+    against an element-by-element count of the allowed matrix."""
+    import bench
+    import oracle
+    for t, w in [(10, 1), (10, 3), (37, 8), (1500, 256)]:
+        assert bench.band_pairs(t, w) == int(oracle.allowed_range(t, t, window=w).sum())
+    spec = inputs.ENCODER_WORKLOADS["varlen8"]
+    lens = inputs.encoder_lengths(spec)
+    assert bench.encoder_pairs(spec) == sum(int(oracle.allowed_range(spec.t, spec.t, q_len=int(n),
+                                                                       kv_len=int(n)).sum()) for n in lens)
+    assert bench.encoder_valid_rows(spec) == int(lens.sum())
