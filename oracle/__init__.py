@@ -12,9 +12,11 @@ from .attention import (  # noqa: F401
     attention,
     attention_head,
     cross_attention,
+    dequantize_q8_0,
     encoder_attention,
     packed_bias,
     qkv_projection,
+    qkv_projection_q8_0,
     range_attention,
     slotmask_attention,
 )

@@ -46,6 +46,13 @@ matmul serves as the library primitive for the dot products.
   value vector: o_i = sum_j e^{s_ij} v_j / (e^{sigma_h} + sum_j e^{s_ij}).
   sigma = -inf is no sink. A row with no allowed key yields 0.
 
+* Q8_0 weights for the projection (edda PR, results table: "Q8_0 decoder").
+  The pages name the GGUF Q8_0 type without defining it; the reading taken is
+  its published layout: each weight row is a run of 34-byte blocks, a
+  little-endian fp16 scale d followed by 32 signed bytes q, and block b of
+  row j holds W[j, 32b + t] = d * q[t]. The projection is then the packed one
+  above with that W, dequantized exactly (a float64 product).
+
 Inputs arrive as fp16 arrays and are widened to float64 exactly. Nothing is
 rounded in between; the output stays float64.
 """
@@ -69,6 +76,31 @@ def packed_bias(b_q: np.ndarray, b_v: np.ndarray) -> np.ndarray:
 def qkv_projection(x: np.ndarray, w_qkv: np.ndarray, b_q: np.ndarray, b_v: np.ndarray) -> np.ndarray:
     """qkv = x . W^T + [b_q | 0 | b_v] in float64.  x [rows, d], W [3d, d] -> [rows, 3d]."""
     return _f64(x) @ _f64(w_qkv).T + packed_bias(b_q, b_v)
+
+
+Q8_0_BLOCK = 32          # weights per block
+Q8_0_BLOCK_BYTES = 34    # fp16 scale + 32 int8
+
+
+def dequantize_q8_0(blocks: np.ndarray, cols: int) -> np.ndarray:
+    """Q8_0 rows (uint8 [rows, cols / 32 * 34]) -> float64 weights [rows, cols]:
+    per block, the fp16 scale times each signed byte."""
+    blocks = np.ascontiguousarray(blocks, dtype=np.uint8)
+    rows = blocks.shape[0]
+    nb = cols // Q8_0_BLOCK
+    if cols % Q8_0_BLOCK or blocks.shape[1] != nb * Q8_0_BLOCK_BYTES:
+        raise ValueError("expected [rows, cols/32 * 34] bytes with cols a multiple of 32")
+    b = blocks.reshape(rows, nb, Q8_0_BLOCK_BYTES)
+    d = b[:, :, :2].copy().view("<f2").astype(np.float64)          # [rows, nb, 1]
+    q = b[:, :, 2:].copy().view(np.int8).astype(np.float64)        # [rows, nb, 32]
+    return (d * q).reshape(rows, cols)
+
+
+def qkv_projection_q8_0(x: np.ndarray, w_blocks: np.ndarray, b_q: np.ndarray, b_v: np.ndarray) -> np.ndarray:
+    """The packed projection with Q8_0 weights: x . W^T + [b_q | 0 | b_v], W
+    dequantized exactly from its blocks. x [rows, d], blocks [3d, d/32 * 34]."""
+    d = np.asarray(x).shape[1]
+    return qkv_projection(x, dequantize_q8_0(w_blocks, d), b_q, b_v)
 
 
 # ----------------------------------------------------------------------------

@@ -33,6 +33,11 @@ Workloads (sizes follow the pages' encoder and decoder):
                    448 keys (432 context positions + the block), 20 heads of 64,
                    per-head sink logits ~ N(0, 1) (seeds 8, 9). Non-causal inside
                    the block by default, causal when the model says so (drafter PR).
+* ``q8_tiny`` / ``q8_verify`` -- the packed projection with Q8_0 weights for
+                   the decoder's verify block (edda PR results table: Q8_0
+                   decoder): 5 x 256 and 80 x 1280 (the 5 beams x 16 rows of
+                   the verify block) rows, q uniform int8, block scales uniform
+                   in [2e-4, 6e-4] (seeds 10, 11).
 * ``verify``    -- decoder block verification over a token tree: 5 beams x
                    (anchor + 15 drafts) = 80 query rows over a 448-slot KV cache,
                    each row limited to its ancestors, plus cross-attention of the
@@ -121,6 +126,59 @@ class DrafterInputs:
     k: np.ndarray      # [beams * (context + block), d_model] float16
     v: np.ndarray      # [beams * (context + block), d_model] float16
     sinks: np.ndarray  # [n_heads] float32 sink logits
+
+
+@dataclasses.dataclass(frozen=True)
+class Q8Spec:
+    name: str
+    rows: int      # decoder rows projected at once
+    d_model: int
+    seed: int
+
+
+Q8_WORKLOADS: Dict[str, Q8Spec] = {
+    "q8_tiny": Q8Spec("q8_tiny", 5, 256, 10),
+    "q8_verify": Q8Spec("q8_verify", 80, 1280, 11),
+}
+
+
+@dataclasses.dataclass
+class Q8Inputs:
+    spec: Q8Spec
+    x: np.ndarray         # [rows, d_model] float16
+    w_blocks: np.ndarray  # [3 * d_model, d_model / 32 * 34] uint8 Q8_0 rows
+    scales: np.ndarray    # [3 * d_model, d_model / 32] float16 (the blocks' scales, for inspection)
+    qs: np.ndarray        # [3 * d_model, d_model] int8 (the blocks' bytes, for inspection)
+    b_q: np.ndarray       # [d_model] float16
+    b_v: np.ndarray       # [d_model] float16
+
+
+def pack_q8_0(scales: np.ndarray, qs: np.ndarray) -> np.ndarray:
+    """Lay out per-block fp16 scales [rows, nb] and int8 values [rows, nb * 32]
+    as Q8_0 rows: per block, the scale's two little-endian bytes, then the
+    32 signed bytes. Byte layout only; no arithmetic on the values."""
+    rows, nb = scales.shape
+    out = np.empty((rows, nb, 34), dtype=np.uint8)
+    out[:, :, :2] = np.ascontiguousarray(scales.astype("<f2")).view(np.uint8).reshape(rows, nb, 2)
+    out[:, :, 2:] = np.ascontiguousarray(qs.astype(np.int8)).view(np.uint8).reshape(rows, nb, 32)
+    return out.reshape(rows, nb * 34)
+
+
+def make_q8_inputs(spec: Q8Spec) -> Q8Inputs:
+    """Random Q8_0 weights drawn directly in their stored form: q uniform in
+    [-127, 127], scales uniform in [2e-4, 6e-4] (the block scale of N(0, 0.02^2)
+    weights, max|w| / 127), rounded to fp16; x ~ N(0, 1); biases ~ N(0, 0.01^2)."""
+    rng = np.random.default_rng(spec.seed)
+    d = spec.d_model
+    if d % 32:
+        raise ValueError("d_model must be a multiple of 32")
+    n = 3 * d
+    qs = rng.integers(-127, 128, size=(n, d)).astype(np.int8)
+    scales = rng.uniform(2e-4, 6e-4, size=(n, d // 32)).astype(np.float16)
+    x = _normal_f16(rng, (spec.rows, d))
+    b_q = _normal_f16(rng, (d,), 0.01)
+    b_v = _normal_f16(rng, (d,), 0.01)
+    return Q8Inputs(spec, x, pack_q8_0(scales, qs), scales, qs, b_q, b_v)
 
 
 def make_drafter_inputs(spec: DrafterSpec) -> DrafterInputs:

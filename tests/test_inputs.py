@@ -116,3 +116,16 @@ def test_bench_pair_counts_match_brute_force():
     assert bench.encoder_pairs(spec) == sum(int(oracle.allowed_range(spec.t, spec.t, q_len=int(n),
                                                                        kv_len=int(n)).sum()) for n in lens)
     assert bench.encoder_valid_rows(spec) == int(lens.sum())
+
+
+def test_q8_inputs_layout_and_determinism():
+    spec = inputs.Q8_WORKLOADS["q8_tiny"]
+    a, b = inputs.make_q8_inputs(spec), inputs.make_q8_inputs(spec)
+    np.testing.assert_array_equal(a.w_blocks, b.w_blocks)
+    d = spec.d_model
+    assert a.w_blocks.shape == (3 * d, d // 32 * 34) and a.w_blocks.dtype == np.uint8
+    # the packed bytes carry exactly the drawn scales and values
+    blk = a.w_blocks.reshape(3 * d, d // 32, 34)
+    np.testing.assert_array_equal(blk[:, :, :2].copy().view("<f2")[..., 0], a.scales)
+    np.testing.assert_array_equal(blk[:, :, 2:].copy().view(np.int8).reshape(3 * d, d), a.qs)
+    assert a.qs.min() >= -127 and a.qs.max() <= 127

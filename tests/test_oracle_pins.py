@@ -481,3 +481,51 @@ def test_sink_edge_cases():
     other = oracle.attention(q, k, v, 2, a, sinks=np.array([60.0, -5.0]))
     np.testing.assert_array_equal(big[:, :64], other[:, :64])
     assert np.abs(big[:, 64:] - other[:, 64:]).max() > 1e-3
+
+
+# ---------------------------------------------------------------------------
+# Q8_0 weights: 34-byte blocks, little-endian fp16 scale then 32 signed bytes
+# ---------------------------------------------------------------------------
+
+def test_q8_0_one_block_by_hand():
+    # scale 0.5 is fp16 0x3800 -> bytes 00 38; q = 1, -2, 3, 127, -128, 0, ...
+    block = bytes([0x00, 0x38, 0x01, 0xFE, 0x03, 0x7F, 0x80] + [0] * 27)
+    assert len(block) == 34
+    w = oracle.dequantize_q8_0(np.frombuffer(block, dtype=np.uint8)[None, :], 32)
+    want = [0.5, -1.0, 1.5, 63.5, -64.0] + [0.0] * 27
+    np.testing.assert_array_equal(w[0], want)
+
+
+def test_q8_0_block_boundaries_and_rows_by_hand():
+    # row 0: block 0 scale 1.0 (0x3C00), all q = 2; block 1 scale -0.25 (0xB400), all q = -4
+    # row 1: block 0 scale 2.0 (0x4000), q[t] = t; block 1 scale 0 -> zeros
+    r0 = bytes([0x00, 0x3C] + [2] * 32 + [0x00, 0xB4] + [0xFC] * 32)
+    r1 = bytes([0x00, 0x40] + list(range(32)) + [0x00, 0x00] + [0x55] * 32)
+    w = oracle.dequantize_q8_0(np.frombuffer(r0 + r1, dtype=np.uint8).reshape(2, 68), 64)
+    np.testing.assert_array_equal(w[0, :32], 2.0)
+    np.testing.assert_array_equal(w[0, 32:], 1.0)      # -0.25 * -4
+    np.testing.assert_array_equal(w[1, :32], 2.0 * np.arange(32))
+    np.testing.assert_array_equal(w[1, 32:], 0.0)
+
+
+def test_q8_0_projection_bruteforce_over_bytes():
+    import struct
+    spec = inputs.Q8Spec("pin", 3, 64, 31)
+    inp = inputs.make_q8_inputs(spec)
+    d = 64
+    got = oracle.qkv_projection_q8_0(inp.x, inp.w_blocks, inp.b_q, inp.b_v)
+    raw = inp.w_blocks
+    for r in range(3):
+        for j in range(3 * d):
+            acc = 0.0
+            for c in range(d):
+                blk = raw[j, (c // 32) * 34:(c // 32) * 34 + 34].tobytes()
+                scale = struct.unpack("<e", blk[:2])[0]
+                q = blk[2 + c % 32]
+                q = q - 256 if q > 127 else q
+                acc += float(inp.x[r, c]) * scale * q
+            if j < d:
+                acc += float(inp.b_q[j])
+            elif j >= 2 * d:
+                acc += float(inp.b_v[j - 2 * d])
+            assert got[r, j] == pytest.approx(acc, rel=1e-12, abs=1e-12)
