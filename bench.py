@@ -44,6 +44,7 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 KERNEL_SOURCES = ["speech_encoder_attention_b200/csrc/flash_attn.cuh",
                   "speech_encoder_attention_b200/csrc/qkv_gemm.cuh",
+                  "speech_encoder_attention_b200/csrc/qkv_q8.cuh",
                   "speech_encoder_attention_b200/csrc/sm100_ptx.cuh",
                   "speech_encoder_attention_b200/csrc/attn_api.cu"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -418,7 +419,63 @@ class DrafterStep:
         return {"query_rows": self.spec.beams * self.spec.t_q}
 
 
+class Q8Step:
+    """The decoder's packed projection with Q8_0 weights (one launch)."""
+
+    def __init__(self, spec: inputs.Q8Spec, device):
+        import torch
+        from speech_encoder_attention_b200 import attn
+        self.attn = attn
+        self.spec = spec
+        inp = inputs.make_q8_inputs(spec)
+        dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+        self.x, self.w, self.bq, self.bv = dev(inp.x), dev(inp.w_blocks), dev(inp.b_q), dev(inp.b_v)
+        d = spec.d_model
+        self.out = torch.empty(spec.rows, 3 * d, dtype=torch.float16, device=device)
+        self.host_x = torch.from_numpy(inp.x).pin_memory()
+        self.host_out = torch.empty(spec.rows, 3 * d, dtype=torch.float16).pin_memory()
+        self.kernels = ["q8_proj"]
+        self.flops = {"q8_proj": qkv_flops(spec.rows, d)}
+        self.bytes = {"q8_proj": inp.w_blocks.nbytes + 2 * spec.rows * d + 2 * spec.rows * 3 * d}
+        self.launches_per_step = 1
+
+    def run(self, events=None):
+        if events:
+            events[0].record()
+        self.attn.attn_qkv_pack_q8_0(self.x, self.w, self.bq, self.bv, out=self.out)
+        if events:
+            events[1].record()
+
+    def run_e2e(self, events=None):
+        if events:
+            events[0].record()
+        self.x.copy_(self.host_x, non_blocking=True)
+        self.run()
+        self.host_out.copy_(self.out, non_blocking=True)
+        if events:
+            events[-1].record()
+
+    @property
+    def h2d_bytes(self):
+        return self.host_x.numel() * 2
+
+    @property
+    def d2h_bytes(self):
+        return self.host_out.numel() * 2
+
+    def total_flops(self):
+        return sum(self.flops.values())
+
+    def total_bytes(self):
+        return sum(self.bytes.values())
+
+    def units(self):
+        return {"rows": self.spec.rows}
+
+
 def make_step(name, device):
+    if name in inputs.Q8_WORKLOADS:
+        return Q8Step(inputs.Q8_WORKLOADS[name], device)
     if name in inputs.ENCODER_WORKLOADS:
         return EncoderStep(inputs.ENCODER_WORKLOADS[name], device)
     if name in inputs.DRAFTER_WORKLOADS:
@@ -474,7 +531,8 @@ def time_oracle(spec, seconds: float = 10.0, max_samples: int = 400):
 
 
 def workload_spec(name):
-    for table in (inputs.ENCODER_WORKLOADS, inputs.VERIFY_WORKLOADS, inputs.DRAFTER_WORKLOADS):
+    for table in (inputs.ENCODER_WORKLOADS, inputs.VERIFY_WORKLOADS, inputs.DRAFTER_WORKLOADS,
+                  inputs.Q8_WORKLOADS):
         if name in table:
             return table[name]
     raise KeyError(name)
@@ -485,6 +543,8 @@ def workload_metric(spec) -> str:
         return METRIC
     if isinstance(spec, inputs.DrafterSpec):
         return "drafter block attention TFLOP/s (HBM-bound; see roofline)"
+    if isinstance(spec, inputs.Q8Spec):
+        return "Q8_0 packed projection TFLOP/s (HBM-bound; see roofline)"
     return "verify+cross attention TFLOP/s (HBM-bound; see roofline)"
 
 
@@ -495,12 +555,17 @@ class SmallOracleStep:
         self.spec = spec
         if isinstance(spec, inputs.DrafterSpec):
             self.inp = inputs.make_drafter_inputs(spec)
+        elif isinstance(spec, inputs.Q8Spec):
+            self.inp = inputs.make_q8_inputs(spec)
         else:
             self.inp = inputs.make_verify_inputs(spec)
 
     def __call__(self, i=0) -> float:
         import oracle
         s, inp = self.spec, self.inp
+        if isinstance(s, inputs.Q8Spec):
+            oracle.qkv_projection_q8_0(inp.x, inp.w_blocks, inp.b_q, inp.b_v)
+            return qkv_flops(s.rows, s.d_model)
         if isinstance(s, inputs.DrafterSpec):
             oracle.range_attention(inp.q, inp.k, inp.v, s.beams, s.t_q, s.t_kv, s.n_heads, causal=s.causal,
                                    sinks=inp.sinks)
@@ -580,6 +645,11 @@ def workload_config(spec):
         if spec.mask == "band":
             cfg["window"] = spec.band
         return cfg
+    if isinstance(spec, inputs.Q8Spec):
+        return {"workload": f"{spec.name}: packed projection of {spec.rows} decoder rows, d_model {spec.d_model}, "
+                            f"Q8_0 weights [{3 * spec.d_model} x {spec.d_model}]",
+                "rows": spec.rows, "d_model": spec.d_model, "weights": "Q8_0 (34-byte blocks)",
+                "l2": "flushed between timed steps (256 MiB write)", "parallelism": "replicas (weak)"}
     if isinstance(spec, inputs.DrafterSpec):
         return {"workload": f"{spec.name}: {spec.beams} beams x {spec.t_q} queries at the end of {spec.t_kv} keys, "
                             f"{'causal' if spec.causal else 'bidirectional'} block, per-head sinks, "
@@ -739,7 +809,7 @@ def parse(argv=None):
     p.add_argument("--impl", choices=["native", "reference"], default="native")
     p.add_argument("--workload", default="windows8",
                    choices=sorted(inputs.ENCODER_WORKLOADS) + sorted(inputs.VERIFY_WORKLOADS)
-                   + sorted(inputs.DRAFTER_WORKLOADS))
+                   + sorted(inputs.DRAFTER_WORKLOADS) + sorted(inputs.Q8_WORKLOADS))
     p.add_argument("--e2e-steps", type=int, default=200)
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--skip-cpu-baseline", action="store_true")

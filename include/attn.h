@@ -118,6 +118,29 @@ attn_status attn_qkv_pack(attn_mat x, const void *w_qkv, const void *b_q, const 
                           int64_t rows, int32_t d_model, attn_mat qkv_out, attn_stream_t stream);
 
 /*
+ * attn_qkv_pack_q8_0 -- the packed QKV projection with Q8_0 weights
+ *   qkv[r, j] = sum_c x[r, c] * W[j, c] + bias[j],  bias = [b_q | 0 | b_v],
+ *   W[j, 32b + t] = d[j, b] * q[j, b, t]
+ * Source: the edda PR's results table (decoder run with Q8_0 weights). The
+ * pages name the GGUF Q8_0 type without defining it; its published layout is
+ * taken: each weight row is d_model/32 blocks of 34 bytes, a little-endian
+ * fp16 scale d followed by 32 signed bytes q (the GGUF tensor's row order).
+ * Meant for the decoder's few rows (a verify block): one CTA per 128 rows x 32
+ * output columns reads each weight row once.
+ *   x        [rows, d_model] fp16, row_stride >= d_model
+ *   w_q8_0   [3*d_model rows of d_model/32 * 34 bytes], contiguous, 16-byte
+ *            aligned (q rows, k rows, v rows)
+ *   b_q, b_v [d_model] fp16 or NULL (zero)
+ *   qkv_out  [rows, 3*d_model] fp16, row_stride >= 3*d_model; must not overlap x or W
+ * d_model must be a positive multiple of 256 (a K step is 8 blocks = 272 bytes,
+ * a multiple of the 16 bytes a tensor-memory-accelerator row needs). Each
+ * weight is dequantized to fp16 (d * q rounded once), the products accumulate
+ * in fp32, the bias is added in fp32 and the result rounded once to fp16.
+ */
+attn_status attn_qkv_pack_q8_0(attn_mat x, const void *w_q8_0, const void *b_q, const void *b_v,
+                               int64_t rows, int32_t d_model, attn_mat qkv_out, attn_stream_t stream);
+
+/*
  * attn_forward -- multi-head flash attention with a mask
  *   o_i = sum_{j in A_i} softmax_j(scale * <q_i, k_j>) v_j     per head
  * A_i by mask.kind: FULL -> all t_kv keys; CHUNK -> keys of the same chunk

@@ -7,6 +7,7 @@ CPU fallback.
 
 The function names match the C entry points:
     attn_qkv_pack(x, w_qkv, b_q, b_v, out=None)        -> qkv
+    attn_qkv_pack_q8_0(x, w_q8_0, b_q, b_v, out=None)  -> qkv
     attn_forward(q, k, v, batch, t_q, t_kv, n_heads, mask=..., out=None) -> out
     attn_forward with sinks=...                          -> attn_forward_sinks
     attn_cross(q, k_enc, v_enc, batch, t_q, t_enc, n_heads, out=None)   -> out
@@ -58,6 +59,8 @@ class AttnMask(ctypes.Structure):
 SIGNATURES = {
     "attn_qkv_pack": (ctypes.c_int, [AttnMat, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                      ctypes.c_int64, ctypes.c_int32, AttnMat, ctypes.c_void_p]),
+    "attn_qkv_pack_q8_0": (ctypes.c_int, [AttnMat, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                          ctypes.c_int64, ctypes.c_int32, AttnMat, ctypes.c_void_p]),
     "attn_forward": (ctypes.c_int, [AttnMat, AttnMat, AttnMat, ctypes.c_int32, ctypes.c_int32,
                                     ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, AttnMask,
                                     ctypes.c_float, AttnMat, ctypes.c_void_p, ctypes.c_size_t,
@@ -156,6 +159,25 @@ def attn_qkv_pack(x, w_qkv, b_q=None, b_v=None, out=None, stream=None):
     st = lib.attn_qkv_pack(_mat(x), _ptr(w_qkv), _ptr(b_q), _ptr(b_v), rows, d, _mat(out),
                            _stream_ptr(stream))
     _check(st, "attn_qkv_pack")
+    return out
+
+
+def attn_qkv_pack_q8_0(x, w_q8_0, b_q=None, b_v=None, out=None, stream=None):
+    """qkv = x . W^T + [b_q | 0 | b_v] with Q8_0 weights: w_q8_0 is a contiguous
+    uint8 CUDA tensor [3*d, d/32*34] (per block: fp16 scale, 32 int8)."""
+    import torch
+    lib = load_library()
+    rows, d = x.shape
+    if w_q8_0.dtype != torch.uint8 or w_q8_0.shape != (3 * d, d // 32 * 34) or not w_q8_0.is_contiguous():
+        raise ValueError("w_q8_0 must be a contiguous [3*d_model, d_model/32*34] uint8 tensor")
+    for b in (b_q, b_v):
+        if b is not None and (b.shape != (d,) or b.dtype != torch.float16 or not b.is_contiguous()):
+            raise ValueError("biases must be contiguous [d_model] fp16 tensors")
+    if out is None:
+        out = torch.empty(rows, 3 * d, dtype=torch.float16, device=x.device)
+    st = lib.attn_qkv_pack_q8_0(_mat(x), _ptr(w_q8_0), _ptr(b_q), _ptr(b_v), rows, d, _mat(out),
+                                _stream_ptr(stream))
+    _check(st, "attn_qkv_pack_q8_0")
     return out
 
 

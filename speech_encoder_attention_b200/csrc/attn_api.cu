@@ -17,6 +17,7 @@
 #include "attn.h"
 #include "flash_attn.cuh"
 #include "qkv_gemm.cuh"
+#include "qkv_q8.cuh"
 #include "sm100_ptx.cuh"
 
 namespace {
@@ -87,6 +88,8 @@ attn_status device_info(DeviceInfo** out) {
     if (cudaGetSymbolAddress(&err, g_error_word) != cudaSuccess) return ATTN_ERR_CUDA;
     if (cudaFuncSetAttribute(sea::gemm::qkv_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              sea::gemm::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(sea::q8::qkv_q8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             sea::q8::SMEM_BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(sea::fa::flash_attn_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              sea::fa::Cfg::SMEM_BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(sea::fa::flash_attn_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -127,6 +130,21 @@ bool encode_2d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, ui
   cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Raw Q8_0 rows as 2-byte units (the 34-byte blocks are not 4-byte aligned;
+// 8 blocks = 272 bytes = 136 units = one box row), no swizzle.
+bool encode_q8_rows(CUtensorMap* m, const void* ptr, uint64_t units_per_row, uint64_t rows, uint32_t box_units,
+                    uint32_t box_rows) {
+  auto enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {units_per_row, rows};
+  cuuint64_t strides[1] = {units_per_row * 2};
+  cuuint32_t box[2] = {box_units, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -386,6 +404,42 @@ attn_status attn_qkv_pack(attn_mat x, const void* w_qkv, const void* b_q, const 
   const int64_t tiles = static_cast<int64_t>(ceil_div(rows, BM)) * ceil_div(n, BN);
   const int grid = static_cast<int>(std::min<int64_t>(tiles, dev->num_sms));
   qkv_gemm_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tx, tw, to, a);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  return ATTN_OK;
+}
+
+attn_status attn_qkv_pack_q8_0(attn_mat x, const void* w_q8_0, const void* b_q, const void* b_v, int64_t rows,
+                               int32_t d_model, attn_mat qkv_out, attn_stream_t stream) {
+  using namespace sea::q8;
+  if (rows <= 0 || rows > INT32_MAX) return ATTN_ERR_INVALID;
+  if (d_model <= 0 || d_model % BKQ != 0 || d_model > 65536) return ATTN_ERR_INVALID;
+  if (!valid_mat(x, d_model) || !valid_mat(qkv_out, 3 * static_cast<int64_t>(d_model))) return ATTN_ERR_INVALID;
+  if (w_q8_0 == nullptr || !aligned16(w_q8_0)) return ATTN_ERR_INVALID;
+  if ((b_q != nullptr && !aligned16(b_q)) || (b_v != nullptr && !aligned16(b_v))) return ATTN_ERR_INVALID;
+  const int64_t n = 3 * static_cast<int64_t>(d_model);
+  const int64_t row_bytes = static_cast<int64_t>(d_model) / QBLOCK * QBLOCK_BYTES;
+  const Range ro = mat_range(qkv_out.ptr, rows, n, qkv_out.row_stride);
+  const Range rw{reinterpret_cast<uintptr_t>(w_q8_0), reinterpret_cast<uintptr_t>(w_q8_0) + n * row_bytes};
+  if (overlaps(ro, mat_range(x.ptr, rows, d_model, x.row_stride)) || overlaps(ro, rw)) return ATTN_ERR_INVALID;
+
+  DeviceInfo* dev = nullptr;
+  if (attn_status st = device_info(&dev); st != ATTN_OK) return st;
+
+  CUtensorMap tx, tw;
+  if (!encode_2d(&tx, x.ptr, d_model, rows, x.row_stride * 2, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_q8_rows(&tw, w_q8_0, row_bytes / 2, n, RAW_ROW_BYTES / 2, BN))
+    return ATTN_ERR_CUDA;
+  Args a{};
+  a.b_q = static_cast<const __half*>(b_q);
+  a.b_v = static_cast<const __half*>(b_v);
+  a.out = static_cast<__half*>(qkv_out.ptr);
+  a.out_stride = qkv_out.row_stride;
+  a.m = static_cast<int>(rows);
+  a.d_model = d_model;
+  a.err = dev->err;
+  a.limit_ns = sea::kDefaultTimeoutNs;
+  const dim3 grid(ceil_div(rows, BM), static_cast<unsigned>(n / BN));
+  qkv_q8_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tx, tw, a);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   return ATTN_OK;
 }

@@ -159,3 +159,17 @@ def test_workspace_size_of_invalid_sizes_is_zero(lib):
     assert lib.attn_workspace_size(0, 80, 1500, 20, 64, 0) == 0
     assert lib.attn_workspace_size(1, 80, 1500, 20, 32, 0) == 0
     assert lib.attn_workspace_size(1, 80, 1500, 20, 64, attn.MASK_CHUNK) == 0
+
+
+@pytest.mark.parametrize("case", [
+    dict(rows=0), dict(d=128), dict(d=384), dict(d=0),          # d_model must be a multiple of 256
+    dict(x=m(0, 256)), dict(x=m(P, 200)), dict(w=0), dict(w=P2 + 2), dict(bq=P3 + 4),
+    dict(out=m(P4, 512)),                                        # row stride < 3*d_model
+    dict(out=m(P2 + 64, 768)),                                   # output overlaps the weights
+])
+def test_qkv_pack_q8_0_rejects_invalid_arguments(lib, case):
+    x = case.get("x", m(P, 256))
+    st = lib.attn_qkv_pack_q8_0(x, ctypes.c_void_p(case.get("w", P2)), ctypes.c_void_p(case.get("bq", P3)),
+                                ctypes.c_void_p(0), case.get("rows", 16), case.get("d", 256),
+                                case.get("out", m(P4, 768)), None)
+    assert st == attn.ATTN_ERR_INVALID
