@@ -313,3 +313,45 @@ def test_many_units_without_keys_back_to_back():
     assert_parity(np.concatenate([got[b * t:(b + 1) * t] for b in sel]), ref, what="empty-unit stress")
     for b, n in enumerate(lens):
         np.testing.assert_array_equal(got[b * t + n:(b + 1) * t], 0.0)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_drafter_projection_reuses_cached_context_rows(causal):
+    """The drafter's packed projection with K/V row reuse, through the public
+    entry points: each beam's packed [context + block, 3d] buffer holds the
+    context rows' q/k/v from an earlier projection (computed once, reused);
+    a step projects only the block's rows into their rows of the buffer and
+    attends from the block's queries over every key of the buffer, with the
+    causal flag and sinks. Must equal the oracle's projection of all rows
+    followed by the same attention."""
+    torch = torch_mod()
+    rng = np.random.default_rng(41 + causal)
+    beams, ctx, block, heads = 3, 150, 16, 4
+    d = heads * 64
+    t_kv = ctx + block
+    w = inputs.random_f16(rng, (3 * d, d), 0.02)
+    bq, bv = inputs.random_f16(rng, (d,), 0.01), inputs.random_f16(rng, (d,), 0.01)
+    x = inputs.random_f16(rng, (beams * t_kv, d))
+    sinks = rng.standard_normal(heads).astype(np.float32)
+    dw, dbq, dbv, ds = to_dev(w), to_dev(bq), to_dev(bv), f32(sinks)
+    cache = torch.zeros(beams * t_kv, 3 * d, dtype=torch.float16, device="cuda")
+    dx = to_dev(x)
+    for b in range(beams):  # context rows: projected once
+        r0 = b * t_kv
+        attn.attn_qkv_pack(dx[r0:r0 + ctx], dw, dbq, dbv, out=cache[r0:r0 + ctx])
+    outs = []
+    for b in range(beams):  # the step: the block's rows only, then attention over the whole buffer
+        r0 = b * t_kv
+        attn.attn_qkv_pack(dx[r0 + ctx:r0 + t_kv], dw, dbq, dbv, out=cache[r0 + ctx:r0 + t_kv])
+        seq = cache[r0:r0 + t_kv]
+        outs.append(attn.attn_forward(seq[ctx:, :d], seq[:, d:2 * d], seq[:, 2 * d:], 1, block, t_kv, heads,
+                                      causal=causal, sinks=ds))
+    torch.cuda.synchronize()
+    got = np.concatenate([to_np64(o) for o in outs])
+    qkv = oracle.qkv_projection(x, w, bq, bv)
+    ref = []
+    for b in range(beams):
+        rows = qkv[b * t_kv:(b + 1) * t_kv]
+        ref.append(oracle.range_attention(rows[ctx:, :d], rows[:, d:2 * d], rows[:, 2 * d:], 1, block, t_kv, heads,
+                                          causal=causal, sinks=sinks))
+    assert_parity(got, np.concatenate(ref), what=f"drafter step causal={causal}")
