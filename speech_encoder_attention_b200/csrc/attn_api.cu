@@ -207,6 +207,25 @@ FaPlan plan_forward(int batch, int t_q, int t_kv, int n_heads, int mask_kind, in
   return pl;
 }
 
+// Launches with programmatic stream serialization: the kernel may start its
+// prologue while the previous kernel in the stream finishes; every kernel of
+// this library waits (griddepcontrol.wait) before it touches global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 bool valid_mat(const attn_mat& m, int64_t cols) {
   return m.ptr != nullptr && aligned16(m.ptr) && m.row_stride >= cols && (m.row_stride % 8) == 0;
 }
@@ -312,26 +331,28 @@ attn_status launch_attention(attn_mat q, attn_mat k, attn_mat v, int32_t batch, 
                    p.kv_lens != nullptr || p.sinks != nullptr;
   const int threads = sea::fa::Cfg::THREADS;
   const int smem = sea::fa::Cfg::SMEM_BYTES;
+  cudaError_t err;
   if (slot) {
     // One unit per CTA (its tile flags need a pass over every row's words).
     if (ext)
-      sea::fa::flash_attn_kernel<true, true><<<p.units, threads, smem, stream>>>(tq, tk, tv, p);
+      err = launch_pdl(sea::fa::flash_attn_kernel<true, true>, dim3(p.units), dim3(threads), smem, stream, tq, tk, tv, p);
     else
-      sea::fa::flash_attn_kernel<true, false><<<p.units, threads, smem, stream>>>(tq, tk, tv, p);
+      err = launch_pdl(sea::fa::flash_attn_kernel<true, false>, dim3(p.units), dim3(threads), smem, stream, tq, tk, tv, p);
   } else {
     // Persistent: Cfg::MIN_BLOCKS CTAs per SM walk the units.
     const int grid = static_cast<int>(std::min<int64_t>(units, int64_t(sea::fa::Cfg::MIN_BLOCKS) * dev->num_sms));
     if (ext)
-      sea::fa::flash_attn_kernel<false, true><<<grid, threads, smem, stream>>>(tq, tk, tv, p);
+      err = launch_pdl(sea::fa::flash_attn_kernel<false, true>, dim3(grid), dim3(threads), smem, stream, tq, tk, tv, p);
     else
-      sea::fa::flash_attn_kernel<false, false><<<grid, threads, smem, stream>>>(tq, tk, tv, p);
+      err = launch_pdl(sea::fa::flash_attn_kernel<false, false>, dim3(grid), dim3(threads), smem, stream, tq, tk, tv, p);
   }
-  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  if (err != cudaSuccess) return ATTN_ERR_CUDA;
   if (pl.kv_splits > 1) {
     const int64_t rows = static_cast<int64_t>(batch) * n_heads * t_q;
-    sea::fa::combine_kernel<<<ceil_div(rows, 8), 256, 0, stream>>>(
-        p.ws_o, p.ws_ml, pl.kv_splits, batch, n_heads, t_q, sinks, p.out, p.out_stride);
-    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    if (launch_pdl(sea::fa::combine_kernel, dim3(ceil_div(rows, 8)), dim3(256), 0, stream,
+                   static_cast<const float*>(p.ws_o), static_cast<const float*>(p.ws_ml), pl.kv_splits, batch,
+                   n_heads, t_q, sinks, p.out, p.out_stride) != cudaSuccess)
+      return ATTN_ERR_CUDA;
   }
   return ATTN_OK;
 }
@@ -403,8 +424,8 @@ attn_status attn_qkv_pack(attn_mat x, const void* w_qkv, const void* b_q, const 
   a.limit_ns = sea::kDefaultTimeoutNs;
   const int64_t tiles = static_cast<int64_t>(ceil_div(rows, BM)) * ceil_div(n, BN);
   const int grid = static_cast<int>(std::min<int64_t>(tiles, dev->num_sms));
-  qkv_gemm_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tx, tw, to, a);
-  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  if (launch_pdl(qkv_gemm_kernel, dim3(grid), dim3(THREADS), SMEM_BYTES, stream, tx, tw, to, a) != cudaSuccess)
+    return ATTN_ERR_CUDA;
   return ATTN_OK;
 }
 
@@ -439,8 +460,8 @@ attn_status attn_qkv_pack_q8_0(attn_mat x, const void* w_q8_0, const void* b_q, 
   a.err = dev->err;
   a.limit_ns = sea::kDefaultTimeoutNs;
   const dim3 grid(ceil_div(rows, BM), static_cast<unsigned>(n / BN));
-  qkv_q8_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tx, tw, a);
-  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  if (launch_pdl(qkv_q8_kernel, grid, dim3(THREADS), SMEM_BYTES, stream, tx, tw, a) != cudaSuccess)
+    return ATTN_ERR_CUDA;
   return ATTN_OK;
 }
 

@@ -290,6 +290,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, Cfg::MIN_BLOCKS)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Everything above touched only this CTA's shared and tensor memory.
+  griddep_wait();
+  griddep_launch_dependents();
   const WaitCtl wc{abort_flag, p.err, p.limit_ns};
   const int srow = (warp & 3) * 32 + lane;  // softmax: row within the tile == TMEM lane
 
@@ -663,6 +666,8 @@ __global__ void __launch_bounds__(256)
     combine_kernel(const float* __restrict__ ws_o, const float* __restrict__ ws_ml, int splits,
                    int batch, int n_heads, int t_q, const float* __restrict__ sinks, __half* __restrict__ out,
                    int64_t out_stride) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int64_t rows = static_cast<int64_t>(batch) * n_heads * t_q;
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (idx >= rows) return;

@@ -125,6 +125,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Everything above touched only this CTA's shared and tensor memory.
+  griddep_wait();
+  griddep_launch_dependents();
   const WaitCtl wc{abort_flag, args.err, args.limit_ns};
 
   if (warp == 0) {

@@ -59,6 +59,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Programmatic dependent launch: wait until the grid this one depends on has
+// completed and its memory is visible (returns at once for a normal launch),
+// then let the next grid in the stream start its own prologue. A dependent
+// grid is launched only once every CTA of this grid has started, so the early
+// trigger cannot take SM resources this grid still needs.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Shared state for cooperative give-up: when any thread's wait expires it sets
 // *abort (shared memory) and the global error word; every other wait in the CTA
 // sees *abort and returns false too, so all roles unwind to the final barrier.
