@@ -35,6 +35,12 @@
  *     no fallback path. A launch failure returns ATTN_ERR_CUDA.
  *   - Device pointers must be 16-byte aligned and row strides multiples of 8
  *     elements (the tensor-memory-accelerator copies need 16-byte strides).
+ *   - Kernels are launched with programmatic stream serialization: each one
+ *     may start its prologue while the previous kernel in the stream finishes,
+ *     and waits for that kernel's completion before touching global memory.
+ *     Ordering on the stream is unchanged for the caller; a caller's own kernel
+ *     that is itself launched programmatically after one of these must wait
+ *     (griddepcontrol.wait) before reading this library's outputs.
  *   - No C++ exception crosses this interface.
  */
 #ifndef SEA_ATTN_H
