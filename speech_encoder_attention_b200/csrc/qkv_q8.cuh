@@ -174,19 +174,23 @@ __global__ void __launch_bounds__(THREADS, 1)
         ok = false;
         break;
       }
-      const uint32_t raw_row = stage_raw(s) + r * RAW_ROW_BYTES;
+      // this thread's two blocks: 34-byte records, so 2-byte loads (plain C++
+      // loads, ordered after the barrier wait, which the compiler may batch)
+      const uint16_t* raw16 = reinterpret_cast<const uint16_t*>(
+          smem + (stage_raw(s) - sbase) + r * RAW_ROW_BYTES + 2 * qq * QBLOCK_BYTES);
       const uint32_t dst_row = stage_b(s) + qq * B_SLICE + r * 128;
+      uint16_t words[2][17];
+#pragma unroll
+      for (int bb = 0; bb < 2; ++bb)
+#pragma unroll
+        for (int i = 0; i < 17; ++i) words[bb][i] = raw16[bb * (QBLOCK_BYTES / 2) + i];
 #pragma unroll
       for (int bb = 0; bb < 2; ++bb) {
-        const uint32_t blk = raw_row + (2 * qq + bb) * QBLOCK_BYTES;  // 2-byte aligned
-        uint16_t dbits;
-        asm volatile("ld.shared.u16 %0, [%1];" : "=h"(dbits) : "r"(blk));
-        const float d = __half2float(__ushort_as_half(dbits));
+        const float d = __half2float(__ushort_as_half(words[bb][0]));
         uint32_t h[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          uint16_t u;
-          asm volatile("ld.shared.u16 %0, [%1];" : "=h"(u) : "r"(blk + 2 + 2 * i));
+          const uint16_t u = words[bb][1 + i];
           const float lo = static_cast<float>(static_cast<int8_t>(u & 0xFF)) * d;
           const float hi = static_cast<float>(static_cast<int8_t>(u >> 8)) * d;
           h[i] = pack_half2(lo, hi);
