@@ -173,3 +173,8 @@ def test_qkv_pack_q8_0_rejects_invalid_arguments(lib, case):
                                 ctypes.c_void_p(0), case.get("rows", 16), case.get("d", 256),
                                 case.get("out", m(P4, 768)), None)
     assert st == attn.ATTN_ERR_INVALID
+
+
+def test_slotmask_slot_limit_is_enforced(lib):
+    mk = attn.AttnMask(); mk.kind = attn.MASK_SLOTMASK; mk.bits = P4 + 0x1000000; mk.words_per_row = 2049
+    assert call_forward(lib, mask=mk, t_kv=65537) == attn.ATTN_ERR_INVALID

@@ -346,3 +346,39 @@ def test_timeout_probe_reports_and_clears():
     assert attn.debug_error_word() == (attn.ATTN_OK, 0)
     # the context is still usable
     test_full_self_attention_lengths(65)
+
+
+# ---------------------------------------------------------------------------
+# maximum sizes and many units
+# ---------------------------------------------------------------------------
+
+def test_slotmask_at_the_slot_limit():
+    """65,536 slots (16 tile-flag words of 32 key tiles): bits spread over the
+    whole range, including the very last slot."""
+    torch = torch_mod()
+    t_q, t_kv, heads = 8, 65536, 1
+    rng = np.random.default_rng(70)
+    q, k, v = rand_qkv(rng, 1, t_q, t_kv, heads)
+    allowed = rng.random((t_q, t_kv)) < 0.002
+    allowed[:, -1] = True
+    allowed[0, :] = False
+    allowed[0, 40000] = True
+    bits = inputs.pack_bits(allowed)
+    got = attn.attn_forward(to_dev(q), to_dev(k), to_dev(v), 1, t_q, t_kv, heads, mask_kind=attn.MASK_SLOTMASK,
+                            bits=to_dev(bits.view(np.int32)))
+    torch.cuda.synchronize()
+    assert_parity(to_np64(got), oracle.attention(q, k, v, heads, allowed), what="slotmask 65536 slots")
+    check_error_word()
+
+
+def test_many_units_per_persistent_cta():
+    """1,024 short sequences: each persistent CTA walks several units."""
+    torch = torch_mod()
+    batch, t, heads = 512, 100, 2
+    rng = np.random.default_rng(71)
+    q, k, v = rand_qkv(rng, batch, t, t, heads)
+    got = attn.attn_forward(to_dev(q), to_dev(k), to_dev(v), batch, t, t, heads)
+    torch.cuda.synchronize()
+    want = oracle_batched(q, k, v, batch, t, t, heads, oracle.allowed_full(t, t))
+    assert_parity(to_np64(got), want, what="512 sequences")
+    check_error_word()
