@@ -776,7 +776,7 @@ def run_gpu(args):
             ent["gbs"] = step.bytes[name] / (per_kernel[k] * 1e-3) / 1e9
         all_kernels[name] = ent
     cpu = None
-    if not args.skip_cpu_baseline:
+    if not args.skip_cpu_baseline and ws == 1:  # the host baseline is an N = 1 figure
         cpu = (time_oracle(spec, seconds=args.cpu_seconds) if is_encoder
                else time_small_oracle(spec, seconds=args.cpu_seconds))
     line = {
