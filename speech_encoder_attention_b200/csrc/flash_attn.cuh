@@ -662,7 +662,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, Cfg::MIN_BLOCKS)
 // Merges the split-KV partials of one (sequence, head, row) per warp:
 //   M = max_s m_s,  L = sum_s l_s 2^(m_s - M) [+ 2^(sink*log2e - M)],
 //   o = sum_s O_s 2^(m_s - M) / L.
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 4)
     combine_kernel(const float* __restrict__ ws_o, const float* __restrict__ ws_ml, int splits,
                    int batch, int n_heads, int t_q, const float* __restrict__ sinks, __half* __restrict__ out,
                    int64_t out_stride) {
@@ -676,21 +676,44 @@ __global__ void __launch_bounds__(256)
   const int h = static_cast<int>((idx / t_q) % n_heads);
   const int b = static_cast<int>(idx / (static_cast<int64_t>(t_q) * n_heads));
   const int64_t stride = rows;  // entries between consecutive splits
+  const float2* ml_p = reinterpret_cast<const float2*>(ws_ml) + idx;
+  const float2* o_p = reinterpret_cast<const float2*>(ws_o + idx * DH) + lane;
+  // Lane j holds split 32g + j's (m, l): one round of loads per 32 splits,
+  // the max and the sum by warp shuffles.
   float mmax = -INFINITY;
-  for (int s = 0; s < splits; ++s) {
-    const float2 ml = reinterpret_cast<const float2*>(ws_ml)[idx + s * stride];
-    if (ml.y > 0.f) mmax = fmaxf(mmax, ml.x);
+  for (int g = 0; g < splits; g += 32) {
+    float m = -INFINITY;
+    if (g + lane < splits) {
+      const float2 ml = ml_p[(g + lane) * stride];
+      if (ml.y > 0.f) m = ml.x;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    mmax = fmaxf(mmax, m);
   }
   float l = 0.f, o0 = 0.f, o1 = 0.f;
   if (mmax != -INFINITY) {
-    for (int s = 0; s < splits; ++s) {
-      const float2 ml = reinterpret_cast<const float2*>(ws_ml)[idx + s * stride];
-      if (!(ml.y > 0.f)) continue;
-      const float w = ex2_approx(ml.x - mmax);
-      l += ml.y * w;
-      const float2 ov = reinterpret_cast<const float2*>(ws_o + (idx + s * stride) * DH)[lane];
-      o0 += ov.x * w;
-      o1 += ov.y * w;
+    for (int g = 0; g < splits; g += 32) {
+      float w = 0.f, lw = 0.f;
+      if (g + lane < splits) {
+        const float2 ml = ml_p[(g + lane) * stride];
+        if (ml.y > 0.f) {
+          w = ex2_approx(ml.x - mmax);
+          lw = ml.y * w;
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, off);
+      l += lw;
+      // each lane's two columns of every split in this group, several loads in flight
+      const int n = min(32, splits - g);
+#pragma unroll 4
+      for (int j = 0; j < n; ++j) {
+        const float wj = __shfl_sync(0xffffffffu, w, j);
+        const float2 ov = o_p[static_cast<int64_t>(g + j) * stride * (DH / 2)];
+        o0 += ov.x * wj;
+        o1 += ov.y * wj;
+      }
     }
     if (sinks != nullptr) l += ex2_approx(__ldg(sinks + h) * kLog2e - mmax);
   }
