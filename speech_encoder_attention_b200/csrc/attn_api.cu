@@ -86,8 +86,12 @@ attn_status device_info(DeviceInfo** out) {
     if (major != 10 || minor != 0) return ATTN_ERR_UNSUPPORTED;
     void* err = nullptr;
     if (cudaGetSymbolAddress(&err, g_error_word) != cudaSuccess) return ATTN_ERR_CUDA;
-    if (cudaFuncSetAttribute(sea::gemm::qkv_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             sea::gemm::SMEM_BYTES) != cudaSuccess ||
+    if (cudaFuncSetAttribute(sea::gemm::qkv_gemm_kernel<sea::gemm::WideTiles>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             sea::gemm::WideTiles::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(sea::gemm::qkv_gemm_kernel<sea::gemm::NarrowTiles>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             sea::gemm::NarrowTiles::SMEM_BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(sea::q8::qkv_q8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              sea::q8::SMEM_BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(sea::fa::flash_attn_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -409,8 +413,15 @@ attn_status attn_qkv_pack(attn_mat x, const void* w_qkv, const void* b_q, const 
 
   CUtensorMap tx, tw, to;
   using namespace sea::gemm;
+  // Tile width by estimated time: waves of 128x256 tiles against waves of
+  // 128x192 tiles, which cost ~0.835 of a wide tile each (measured on B200).
+  const int64_t m_tiles = ceil_div(rows, BM);
+  const int64_t waves_wide = (m_tiles * ceil_div(n, WideTiles::BN) + dev->num_sms - 1) / dev->num_sms;
+  const int64_t waves_narrow = (m_tiles * ceil_div(n, NarrowTiles::BN) + dev->num_sms - 1) / dev->num_sms;
+  const bool narrow = n % NarrowTiles::BN == 0 && waves_narrow * 835 < waves_wide * 1000;
+  const int bn = narrow ? NarrowTiles::BN : WideTiles::BN;
   if (!encode_2d(&tx, x.ptr, d_model, rows, x.row_stride * 2, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_2d(&tw, w_qkv, d_model, n, static_cast<uint64_t>(d_model) * 2, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&tw, w_qkv, d_model, n, static_cast<uint64_t>(d_model) * 2, BK, bn, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_2d(&to, qkv_out.ptr, n, rows, qkv_out.row_stride * 2, EPI_COLS, 32, CU_TENSOR_MAP_SWIZZLE_64B))
     return ATTN_ERR_CUDA;
   Args a{};
@@ -422,10 +433,14 @@ attn_status attn_qkv_pack(attn_mat x, const void* w_qkv, const void* b_q, const 
   a.d_model = d_model;
   a.err = dev->err;
   a.limit_ns = sea::kDefaultTimeoutNs;
-  const int64_t tiles = static_cast<int64_t>(ceil_div(rows, BM)) * ceil_div(n, BN);
+  const int64_t tiles = m_tiles * ceil_div(n, bn);
   const int grid = static_cast<int>(std::min<int64_t>(tiles, dev->num_sms));
-  if (launch_pdl(qkv_gemm_kernel, dim3(grid), dim3(THREADS), SMEM_BYTES, stream, tx, tw, to, a) != cudaSuccess)
-    return ATTN_ERR_CUDA;
+  const cudaError_t err =
+      narrow ? launch_pdl(qkv_gemm_kernel<NarrowTiles>, dim3(grid), dim3(THREADS), NarrowTiles::SMEM_BYTES, stream, tx,
+                          tw, to, a)
+             : launch_pdl(qkv_gemm_kernel<WideTiles>, dim3(grid), dim3(THREADS), WideTiles::SMEM_BYTES, stream, tx, tw,
+                          to, a);
+  if (err != cudaSuccess) return ATTN_ERR_CUDA;
   return ATTN_OK;
 }
 
