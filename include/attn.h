@@ -59,7 +59,7 @@ typedef struct CUstream_st *attn_stream_t;
 typedef enum {
   ATTN_OK = 0,
   ATTN_ERR_INVALID = 1,     /* bad argument; nothing was launched */
-  ATTN_ERR_UNSUPPORTED = 2, /* valid request this build does not serve (e.g. no sm_100 device) */
+  ATTN_ERR_UNSUPPORTED = 2, /* valid request this library does not serve (e.g. no sm_100 device) */
   ATTN_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
   ATTN_ERR_TIMEOUT = 4      /* a kernel's bounded wait expired (see attn_debug_error_word) */
 } attn_status;
