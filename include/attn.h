@@ -245,6 +245,31 @@ const char *attn_status_string(attn_status status);
 attn_status attn_debug_error_word(attn_stream_t stream, uint32_t *word_out);
 
 /*
+ * attn_debug_plan -- the host-side launch plan, without a device: what
+ * attn_forward / attn_qkv_pack would choose on a GPU with num_sms SMs.
+ *   seg_len, tiles_per_seg, q_tiles: the query-tile schedule (CHUNK: segments
+ *     of whole chunks; otherwise one segment of t_q rows)
+ *   kv_splits, kv_tiles_per_split: the key split (1 = none); units = work units
+ *   workspace_bytes: what attn_workspace_size would report for that device
+ *   proj_tile_n: the projection's output tile width for proj_rows rows of
+ *     d_model (256 or 192; 0 when proj_rows or d_model is 0)
+ * Pure host arithmetic (no CUDA call). Returns ATTN_ERR_INVALID for
+ * non-positive sizes or SM count, an unknown mask kind or CHUNK without a
+ * positive chunk_len.
+ */
+typedef struct {
+  int32_t seg_len, tiles_per_seg, q_tiles;
+  int32_t kv_splits, kv_tiles_per_split;
+  int32_t proj_tile_n;
+  int64_t units;
+  size_t workspace_bytes;
+} attn_plan_info;
+
+attn_status attn_debug_plan(int32_t batch, int32_t t_q, int32_t t_kv, int32_t n_heads, int32_t mask_kind,
+                            int32_t chunk_len, int32_t num_sms, int64_t proj_rows, int32_t d_model,
+                            attn_plan_info *out);
+
+/*
  * attn_debug_timeout_probe -- launches one tiny kernel that waits on a barrier
  * nothing will ever complete, with a limit of limit_ns nanoseconds (1e3..1e9).
  * The kernel gives up, records the timeout in the error word and returns, so

@@ -55,6 +55,19 @@ class AttnMask(ctypes.Structure):
     ]
 
 
+class AttnPlanInfo(ctypes.Structure):
+    _fields_ = [
+        ("seg_len", ctypes.c_int32),
+        ("tiles_per_seg", ctypes.c_int32),
+        ("q_tiles", ctypes.c_int32),
+        ("kv_splits", ctypes.c_int32),
+        ("kv_tiles_per_split", ctypes.c_int32),
+        ("proj_tile_n", ctypes.c_int32),
+        ("units", ctypes.c_int64),
+        ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
 # (name, restype, argtypes) of every exported entry point.
 SIGNATURES = {
     "attn_qkv_pack": (ctypes.c_int, [AttnMat, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
@@ -79,6 +92,8 @@ SIGNATURES = {
     "attn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "attn_debug_error_word": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_uint32)]),
     "attn_debug_timeout_probe": (ctypes.c_int, [ctypes.c_int64, ctypes.c_void_p]),
+    "attn_debug_plan": (ctypes.c_int, [ctypes.c_int32] * 7 + [ctypes.c_int64, ctypes.c_int32,
+                                                              ctypes.POINTER(AttnPlanInfo)]),
 }
 
 _lib = None
@@ -289,3 +304,13 @@ def debug_error_word(stream=None):
 
 def debug_timeout_probe(limit_ns: int, stream=None) -> int:
     return load_library().attn_debug_timeout_probe(int(limit_ns), _stream_ptr(stream))
+
+
+def debug_plan(batch, t_q, t_kv, n_heads, mask_kind=MASK_FULL, chunk_len=0, num_sms=148, proj_rows=0,
+               d_model=0) -> dict:
+    """The launch plan the library would choose on a GPU with num_sms SMs (host arithmetic only)."""
+    info = AttnPlanInfo()
+    st = load_library().attn_debug_plan(batch, t_q, t_kv, n_heads, mask_kind, chunk_len, num_sms, proj_rows,
+                                        d_model, ctypes.byref(info))
+    _check(st, "attn_debug_plan")
+    return {name: getattr(info, name) for name, _ in AttnPlanInfo._fields_}

@@ -230,6 +230,18 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// Projection tile width by estimated time: waves of 128x256 tiles against
+// waves of 128x192 tiles, which cost ~0.835 of a wide tile each (measured on
+// B200).
+int gemm_tile_n(int64_t rows, int64_t n, int num_sms) {
+  using namespace sea::gemm;
+  const int64_t m_tiles = ceil_div(rows, BM);
+  const int64_t waves_wide = (m_tiles * ceil_div(n, WideTiles::BN) + num_sms - 1) / num_sms;
+  const int64_t waves_narrow = (m_tiles * ceil_div(n, NarrowTiles::BN) + num_sms - 1) / num_sms;
+  const bool narrow = n % NarrowTiles::BN == 0 && waves_narrow * 835 < waves_wide * 1000;
+  return narrow ? NarrowTiles::BN : WideTiles::BN;
+}
+
 bool valid_mat(const attn_mat& m, int64_t cols) {
   return m.ptr != nullptr && aligned16(m.ptr) && m.row_stride >= cols && (m.row_stride % 8) == 0;
 }
@@ -413,13 +425,9 @@ attn_status attn_qkv_pack(attn_mat x, const void* w_qkv, const void* b_q, const 
 
   CUtensorMap tx, tw, to;
   using namespace sea::gemm;
-  // Tile width by estimated time: waves of 128x256 tiles against waves of
-  // 128x192 tiles, which cost ~0.835 of a wide tile each (measured on B200).
   const int64_t m_tiles = ceil_div(rows, BM);
-  const int64_t waves_wide = (m_tiles * ceil_div(n, WideTiles::BN) + dev->num_sms - 1) / dev->num_sms;
-  const int64_t waves_narrow = (m_tiles * ceil_div(n, NarrowTiles::BN) + dev->num_sms - 1) / dev->num_sms;
-  const bool narrow = n % NarrowTiles::BN == 0 && waves_narrow * 835 < waves_wide * 1000;
-  const int bn = narrow ? NarrowTiles::BN : WideTiles::BN;
+  const int bn = gemm_tile_n(rows, n, dev->num_sms);
+  const bool narrow = bn == NarrowTiles::BN;
   if (!encode_2d(&tx, x.ptr, d_model, rows, x.row_stride * 2, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_2d(&tw, w_qkv, d_model, n, static_cast<uint64_t>(d_model) * 2, BK, bn, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_2d(&to, qkv_out.ptr, n, rows, qkv_out.row_stride * 2, EPI_COLS, 32, CU_TENSOR_MAP_SWIZZLE_64B))
@@ -550,6 +558,26 @@ attn_status attn_debug_error_word(attn_stream_t stream, uint32_t* word_out) {
   if (cudaMemcpy(dev->err, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return ATTN_ERR_CUDA;
   if (word_out) *word_out = w;
   return w ? ATTN_ERR_TIMEOUT : ATTN_OK;
+}
+
+attn_status attn_debug_plan(int32_t batch, int32_t t_q, int32_t t_kv, int32_t n_heads, int32_t mask_kind,
+                            int32_t chunk_len, int32_t num_sms, int64_t proj_rows, int32_t d_model,
+                            attn_plan_info* out) {
+  if (out == nullptr || batch <= 0 || t_q <= 0 || t_kv <= 0 || n_heads <= 0 || num_sms <= 0) return ATTN_ERR_INVALID;
+  if (mask_kind < ATTN_MASK_FULL || mask_kind > ATTN_MASK_BAND) return ATTN_ERR_INVALID;
+  if (mask_kind == ATTN_MASK_CHUNK && chunk_len <= 0) return ATTN_ERR_INVALID;
+  const int kind = (mask_kind == ATTN_MASK_CHUNK && chunk_len >= t_q) ? ATTN_MASK_FULL : mask_kind;
+  const FaPlan pl = plan_forward(batch, t_q, t_kv, n_heads, kind, chunk_len, num_sms);
+  out->seg_len = pl.seg_len;
+  out->tiles_per_seg = pl.tiles_per_seg;
+  out->q_tiles = pl.q_tiles;
+  out->kv_splits = pl.kv_splits;
+  out->kv_tiles_per_split = pl.kv_tiles_per_split;
+  out->units = static_cast<int64_t>(batch) * n_heads * pl.q_tiles * pl.kv_splits;
+  out->workspace_bytes = pl.ws_bytes;
+  out->proj_tile_n = (proj_rows > 0 && d_model > 0) ? gemm_tile_n(proj_rows, 3 * static_cast<int64_t>(d_model), num_sms)
+                                                    : 0;
+  return ATTN_OK;
 }
 
 attn_status attn_debug_timeout_probe(int64_t limit_ns, attn_stream_t stream) {

@@ -178,3 +178,69 @@ def test_qkv_pack_q8_0_rejects_invalid_arguments(lib, case):
 def test_slotmask_slot_limit_is_enforced(lib):
     mk = attn.AttnMask(); mk.kind = attn.MASK_SLOTMASK; mk.bits = P4 + 0x1000000; mk.words_per_row = 2049
     assert call_forward(lib, mask=mk, t_kv=65537) == attn.ATTN_ERR_INVALID
+
+
+# ---------------------------------------------------------------------------
+# host launch plan (no device needed)
+# ---------------------------------------------------------------------------
+
+def test_plan_of_the_benchmarked_and_one_window_steps(lib):
+    p = attn.debug_plan(8, 1500, 1500, 20, proj_rows=12000, d_model=1280)
+    assert (p["q_tiles"], p["kv_splits"], p["units"], p["workspace_bytes"]) == (12, 1, 8 * 20 * 12, 0)
+    # 94 x 15 wide tiles = 9.53 waves against 94 x 20 narrow ones = 12.7: wide
+    assert p["proj_tile_n"] == 256
+    # 12 x 15 = 180 wide tiles = 2 waves, 12 x 20 = 240 narrow = 2 waves of smaller tiles: narrow
+    assert attn.debug_plan(1, 1500, 1500, 20, proj_rows=1500, d_model=1280)["proj_tile_n"] == 192
+
+
+@pytest.mark.parametrize("t,clen", [(2325, 200), (517, 7), (517, 128), (517, 150), (300, 1)])
+def test_plan_chunk_segments_are_whole_chunks(lib, t, clen):
+    p = attn.debug_plan(1, t, t, 2, attn.MASK_CHUNK, clen)
+    seg = clen if clen >= 128 else (128 // clen) * clen  # one chunk, or as many whole chunks as fit 128 rows
+    assert p["seg_len"] == seg and p["seg_len"] % clen == 0
+    assert p["tiles_per_seg"] == -(-seg // 128)
+    assert p["q_tiles"] == -(-t // seg) * p["tiles_per_seg"]
+    assert p["kv_splits"] == 1 and p["workspace_bytes"] == 0  # CHUNK tiles already fill the GPU
+
+
+def test_plan_chunk_at_least_the_sequence_is_full(lib):
+    a = attn.debug_plan(2, 300, 300, 2, attn.MASK_CHUNK, 300)
+    b = attn.debug_plan(2, 300, 300, 2, attn.MASK_FULL)
+    assert a == b
+
+
+@pytest.mark.parametrize("kind,t_q,t_kv,heads,sms", [
+    (attn.MASK_SLOTMASK, 80, 448, 20, 148),   # the verify block: 4 key tiles
+    (attn.MASK_FULL, 80, 1500, 20, 148),      # cross-attention: 12 key tiles
+    (attn.MASK_BAND, 16, 448, 5, 148),
+    (attn.MASK_FULL, 80, 1500, 20, 64),
+])
+def test_plan_splits_short_query_blocks(lib, kind, t_q, t_kv, heads, sms):
+    p = attn.debug_plan(1, t_q, t_kv, heads, kind, num_sms=sms)
+    base = heads * -(-t_q // 128)
+    n_kv = -(-t_kv // 128)
+    assert base * 2 <= sms  # these cases qualify for a split
+    want = min(n_kv, max(1, sms // base))
+    per = -(-n_kv // want)
+    splits = -(-n_kv // per)
+    assert (p["kv_splits"], p["kv_tiles_per_split"]) == (splits, per)
+    assert p["kv_splits"] * p["kv_tiles_per_split"] >= n_kv > (p["kv_splits"] - 1) * p["kv_tiles_per_split"]
+    assert p["units"] == base * splits
+    rows = splits * heads * t_q
+    assert p["workspace_bytes"] == rows * 64 * 4 + rows * 2 * 4  # partial O, then (m, l)
+
+
+def test_plan_does_not_split_when_units_fill_the_gpu(lib):
+    p = attn.debug_plan(1, 80, 1500, 80, num_sms=148)  # 80 units: more than half of 148
+    assert p["kv_splits"] == 1 and p["workspace_bytes"] == 0
+    p = attn.debug_plan(1, 80, 100, 20, num_sms=148)    # a single key tile: nothing to split
+    assert p["kv_splits"] == 1
+
+
+def test_plan_rejects_invalid_requests(lib):
+    info = attn.AttnPlanInfo()
+    assert lib.attn_debug_plan(0, 1, 1, 1, 0, 0, 148, 0, 0, ctypes.byref(info)) == attn.ATTN_ERR_INVALID
+    assert lib.attn_debug_plan(1, 1, 1, 1, 0, 0, 0, 0, 0, ctypes.byref(info)) == attn.ATTN_ERR_INVALID
+    assert lib.attn_debug_plan(1, 1, 1, 1, 9, 0, 148, 0, 0, ctypes.byref(info)) == attn.ATTN_ERR_INVALID
+    assert lib.attn_debug_plan(1, 8, 8, 1, attn.MASK_CHUNK, 0, 148, 0, 0, ctypes.byref(info)) == attn.ATTN_ERR_INVALID
+    assert lib.attn_debug_plan(1, 1, 1, 1, 0, 0, 148, 0, 0, None) == attn.ATTN_ERR_INVALID
