@@ -24,6 +24,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import re
 import os
 import socket
 import subprocess
@@ -86,11 +87,21 @@ def encoder_valid_rows(spec: inputs.EncoderSpec) -> int:
     return int(lens.sum()) if lens is not None else spec.batch * spec.t
 
 
+def _strip_comments(src: str) -> str:
+    """C/C++ source without its comments and blank lines (string literals in
+    these files hold no comment markers)."""
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+
+
 def kernel_source_hash() -> str:
+    """Hash of the kernel and launch code (comments excluded): stored ncu
+    counters are valid while it is unchanged."""
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+            h.update(_strip_comments(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -8,7 +8,10 @@
 // window, the query's own chunk for the higgs chunked encoder
 // ("higgs-audio-v3-stt GGUF", "Architecture note (chunked encoder)"), and the
 // query row's ancestor slots for the token-tree verify pass (edda PR
-// description, beam search over a token-tree KV cache).
+// description, beam search over a token-tree KV cache). The range family
+// (FULL, CHUNK, BAND) also takes per-sequence lengths and a causal flag, and
+// per-head sinks join the normaliser (drafter PR: causal flag, sliding window,
+// attention sinks); those options are a separate compile-time variant (EXT).
 //
 // Work unit: one 128-row query tile of one (sequence, head) against a range
 // of 128-row key/value tiles (the whole sequence, the tile's chunk, or one
@@ -32,7 +35,8 @@
 // SLOTMASK skips key tiles whose mask words are zero for every row of the CTA.
 // Split-KV: for short query blocks the key range is split over units; each
 // writes unnormalised O with its m and l to the workspace and a combine kernel
-// merges them.
+// merges them. Every kernel here waits (griddepcontrol) after its prologue, so
+// programmatic launches overlap that prologue with the previous kernel.
 #pragma once
 
 #include "sm100_ptx.cuh"
