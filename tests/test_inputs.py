@@ -129,3 +129,17 @@ def test_q8_inputs_layout_and_determinism():
     np.testing.assert_array_equal(blk[:, :, :2].copy().view("<f2")[..., 0], a.scales)
     np.testing.assert_array_equal(blk[:, :, 2:].copy().view(np.int8).reshape(3 * d, d), a.qs)
     assert a.qs.min() >= -127 and a.qs.max() <= 127
+
+
+def test_kernel_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
+    """Stored ncu counters stay valid across comment edits, not code edits."""
+    import bench
+    src = tmp_path / "k.cuh"
+    src.write_text("// header\nint f(int x) {  // trailing\n  return x + 1; /* note */\n}\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "KERNEL_SOURCES", ["k.cuh"])
+    h0 = bench.kernel_source_hash()
+    src.write_text("// a different header\n/* block\n comment */\nint f(int x) {\n  return x + 1;\n}\n")
+    assert bench.kernel_source_hash() == h0
+    src.write_text("int f(int x) {\n  return x + 2;\n}\n")
+    assert bench.kernel_source_hash() != h0
