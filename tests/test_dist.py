@@ -77,3 +77,18 @@ def test_reference_arm_prints_one_line(monkeypatch, capsys):
     line = json.loads(out[0])
     assert line["impl"] == "reference" and line["unit"] == "TFLOP/s" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+@pytest.mark.parametrize("workload,metric_word", [("q8_tiny", "Q8_0"), ("drafter", "drafter"), ("verify", "verify")])
+def test_reference_arm_small_workloads(monkeypatch, capsys, workload, metric_word):
+    """The whole-step oracle of the decoder-side workloads, same line format."""
+    import json
+
+    import bench
+    for key in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        monkeypatch.delenv(key, raising=False)
+    assert bench.main(["--impl", "reference", "--workload", workload, "--steps", "1", "--warmup", "0"]) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and metric_word in line["metric"] and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle"
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
