@@ -223,6 +223,57 @@ def test_chunk_len_one_returns_values_and_long_chunk_is_full():
         np.testing.assert_array_equal(oracle.attention(q, k, v, 1, oracle.allowed_chunk(t, clen)), full)
 
 
+def _window_rows_bruteforce(qkv, rows, n_heads, d):
+    """Pure-Python attention of the frames `rows` (global row indices) among
+    themselves only, from a packed qkv matrix: the definition of one window (or
+    one chunk) encoded on its own."""
+    q = [qkv[r, :d].tolist() for r in rows]
+    k = [qkv[r, d:2 * d].tolist() for r in rows]
+    v = [qkv[r, 2 * d:].tolist() for r in rows]
+    return _brute_force(q, k, v, [list(range(len(rows)))] * len(rows), n_heads)
+
+
+def test_encoder_windows_attend_only_within_themselves():
+    """Each window of a batch is its own bidirectional sequence: the batched
+    encoder path equals, window by window, brute-force attention over that
+    window's frames alone (windows carry different offsets, so a window that
+    saw another window's keys would differ)."""
+    batch, t, d, heads = 3, 13, 128, 2
+    spec = inputs.EncoderSpec("t", batch, t, d, heads, "full", 0, 21, True)
+    inp = inputs.make_encoder_inputs(spec)
+    got = oracle.encoder_attention(inp.x, inp.w_qkv, inp.b_q, inp.b_v, batch, t, heads)
+    qkv = oracle.qkv_projection(inp.x, inp.w_qkv, inp.b_q, inp.b_v)
+    for b in range(batch):
+        rows = list(range(b * t, (b + 1) * t))
+        want = _window_rows_bruteforce(qkv, rows, heads, d)
+        np.testing.assert_allclose(got[b * t:(b + 1) * t], want, rtol=1e-12, atol=1e-13)
+    # the same frames run as one long sequence give a different answer
+    whole = _window_rows_bruteforce(qkv, list(range(t)) + list(range(t, 2 * t)), heads, d)
+    assert np.abs(whole[:t] - got[:t]).max() > 1e-4
+
+
+def test_encoder_chunk_mode_equals_independent_chunks():
+    """CHUNK(len) through the batched encoder path: every chunk of every window
+    (chunks restart at each window's frame 0, the last one short) equals
+    brute-force attention over that chunk's frames alone."""
+    batch, t, clen, d, heads = 2, 12, 5, 128, 2
+    spec = inputs.EncoderSpec("t", batch, t, d, heads, "chunk", clen, 22, True)
+    inp = inputs.make_encoder_inputs(spec)
+    got = oracle.encoder_attention(inp.x, inp.w_qkv, inp.b_q, inp.b_v, batch, t, heads,
+                                   mask="chunk", chunk_len=clen)
+    qkv = oracle.qkv_projection(inp.x, inp.w_qkv, inp.b_q, inp.b_v)
+    spans = []
+    for b in range(batch):
+        for c0 in range(0, t, clen):
+            spans.append(list(range(b * t + c0, b * t + min(c0 + clen, t))))
+    assert [len(s) for s in spans] == [5, 5, 2, 5, 5, 2]
+    for rows in spans:
+        want = _window_rows_bruteforce(qkv, rows, heads, d)
+        np.testing.assert_allclose(got[rows], want, rtol=1e-12, atol=1e-13)
+    full = oracle.encoder_attention(inp.x, inp.w_qkv, inp.b_q, inp.b_v, batch, t, heads)
+    assert np.abs(full - got).max() > 1e-4
+
+
 def test_chunk_boundaries_by_hand():
     a = oracle.allowed_chunk(7, 3)
     want = np.array([[1, 1, 1, 0, 0, 0, 0],
