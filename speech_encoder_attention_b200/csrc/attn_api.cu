@@ -16,6 +16,7 @@
 
 #include "attn.h"
 #include "flash_attn.cuh"
+#include "flash_range.cuh"
 #include "qkv_gemm.cuh"
 #include "qkv_q8.cuh"
 #include "sm100_ptx.cuh"
@@ -92,6 +93,8 @@ attn_status device_info(DeviceInfo** out) {
         cudaFuncSetAttribute(sea::gemm::qkv_gemm_kernel<sea::gemm::NarrowTiles>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              sea::gemm::NarrowTiles::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(sea::gemm::qkv_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             sea::gemm::PairShape::SMEM_BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(sea::q8::qkv_q8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              sea::q8::SMEM_BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(sea::fa::flash_attn_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -101,7 +104,11 @@ attn_status device_info(DeviceInfo** out) {
         cudaFuncSetAttribute(sea::fa::flash_attn_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              sea::fa::Cfg::SMEM_BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(sea::fa::flash_attn_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             sea::fa::Cfg::SMEM_BYTES) != cudaSuccess)
+                             sea::fa::Cfg::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(sea::fr::flash_range_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             sea::fr::Cfg::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(sea::fr::flash_range_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             sea::fr::Cfg::SMEM_BYTES) != cudaSuccess)
       return ATTN_ERR_CUDA;
     d.num_sms = sms;
     d.err = static_cast<uint32_t*>(err);
@@ -214,27 +221,58 @@ FaPlan plan_forward(int batch, int t_q, int t_kv, int n_heads, int mask_kind, in
 // Launches with programmatic stream serialization: the kernel may start its
 // prologue while the previous kernel in the stream finishes; every kernel of
 // this library waits (griddepcontrol.wait) before it touches global memory.
+// cluster_x > 1 launches thread-block clusters of that many CTAs along x.
 template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
-                       Args&&... args) {
+cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                               unsigned cluster_x, Args&&... args) {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  unsigned n = 1;
+  if (cluster_x > 1) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster_x;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    n = 2;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = n;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+  return launch_pdl_cluster(kernel, grid, block, smem, stream, 1u, std::forward<Args>(args)...);
+}
+
+// The range masks (FULL, CHUNK, BAND and their options) run on the one-CTA-
+// per-SM kernel of flash_range.cuh when set, else on flash_attn.cuh's.
+#ifndef SEA_RANGE_KERNEL_V2
+#define SEA_RANGE_KERNEL_V2 0
+#endif
+constexpr bool kRangeKernelV2 = SEA_RANGE_KERNEL_V2 != 0;
+
+// Row counts from which the projection runs on CTA pairs (256 x 256 tiles,
+// cta_group::2): large enough that the pair tiles fill the GPU.
+#ifndef SEA_PAIR_MIN_ROWS
+#define SEA_PAIR_MIN_ROWS (1 << 30)
+#endif
+constexpr int64_t kPairMinRows = SEA_PAIR_MIN_ROWS;
+constexpr int kPairTileN = 512;  // plan code for the pair kernel (tile 256 rows x 256 columns)
 
 // Projection tile width by estimated time: waves of 128x256 tiles against
 // waves of 128x192 tiles, which cost ~0.835 of a wide tile each (measured on
 // B200).
 int gemm_tile_n(int64_t rows, int64_t n, int num_sms) {
   using namespace sea::gemm;
+  if (rows >= kPairMinRows && n % PairShape::BN == 0) return kPairTileN;
   const int64_t m_tiles = ceil_div(rows, BM);
   const int64_t waves_wide = (m_tiles * ceil_div(n, WideTiles::BN) + num_sms - 1) / num_sms;
   const int64_t waves_narrow = (m_tiles * ceil_div(n, NarrowTiles::BN) + num_sms - 1) / num_sms;
@@ -246,10 +284,11 @@ bool valid_mat(const attn_mat& m, int64_t cols) {
   return m.ptr != nullptr && aligned16(m.ptr) && m.row_stride >= cols && (m.row_stride % 8) == 0;
 }
 
-attn_status launch_attention(attn_mat q, attn_mat k, attn_mat v, int32_t batch, int32_t t_q, int32_t t_kv,
-                             int32_t n_heads, int32_t head_dim, attn_mask mask, const float* sinks, float scale,
-                             attn_mat out, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
-  // ---- validation (host only, before any CUDA call) ----
+// Argument checks of the attention entry points: pure host arithmetic on the
+// arguments, no CUDA call. ATTN_OK or ATTN_ERR_INVALID.
+attn_status validate_attention(attn_mat q, attn_mat k, attn_mat v, int32_t batch, int32_t t_q, int32_t t_kv,
+                               int32_t n_heads, int32_t head_dim, const attn_mask& mask, const float* sinks,
+                               float scale, attn_mat out, const void* workspace, size_t workspace_bytes) {
   if (batch <= 0 || t_q <= 0 || t_kv <= 0 || n_heads <= 0) return ATTN_ERR_INVALID;
   if (head_dim != sea::fa::DH) return ATTN_ERR_INVALID;
   if (batch > 65535 || n_heads > 65535) return ATTN_ERR_INVALID;
@@ -284,6 +323,17 @@ attn_status launch_attention(attn_mat q, attn_mat k, attn_mat v, int32_t batch, 
     return ATTN_ERR_INVALID;
   if (workspace != nullptr && !aligned16(workspace)) return ATTN_ERR_INVALID;
   if (workspace == nullptr && workspace_bytes != 0) return ATTN_ERR_INVALID;
+  return ATTN_OK;
+}
+
+attn_status launch_attention(attn_mat q, attn_mat k, attn_mat v, int32_t batch, int32_t t_q, int32_t t_kv,
+                             int32_t n_heads, int32_t head_dim, attn_mask mask, const float* sinks, float scale,
+                             attn_mat out, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (attn_status st = validate_attention(q, k, v, batch, t_q, t_kv, n_heads, head_dim, mask, sinks, scale, out,
+                                          workspace, workspace_bytes);
+      st != ATTN_OK)
+    return st;
+  const int64_t cols = static_cast<int64_t>(n_heads) * head_dim;
 
   DeviceInfo* dev = nullptr;
   if (attn_status st = device_info(&dev); st != ATTN_OK) return st;
@@ -354,6 +404,16 @@ attn_status launch_attention(attn_mat q, attn_mat k, attn_mat v, int32_t batch, 
       err = launch_pdl(sea::fa::flash_attn_kernel<true, true>, dim3(p.units), dim3(threads), smem, stream, tq, tk, tv, p);
     else
       err = launch_pdl(sea::fa::flash_attn_kernel<true, false>, dim3(p.units), dim3(threads), smem, stream, tq, tk, tv, p);
+  } else if (kRangeKernelV2) {
+    // Persistent: one CTA per SM walks the units.
+    using FR = sea::fr::Cfg;
+    const int grid = static_cast<int>(std::min<int64_t>(units, dev->num_sms));
+    if (ext)
+      err = launch_pdl(sea::fr::flash_range_kernel<true>, dim3(grid), dim3(FR::THREADS), FR::SMEM_BYTES, stream, tq, tk,
+                       tv, p);
+    else
+      err = launch_pdl(sea::fr::flash_range_kernel<false>, dim3(grid), dim3(FR::THREADS), FR::SMEM_BYTES, stream, tq,
+                       tk, tv, p);
   } else {
     // Persistent: Cfg::MIN_BLOCKS CTAs per SM walk the units.
     const int grid = static_cast<int>(std::min<int64_t>(units, int64_t(sea::fa::Cfg::MIN_BLOCKS) * dev->num_sms));
@@ -427,9 +487,13 @@ attn_status attn_qkv_pack(attn_mat x, const void* w_qkv, const void* b_q, const 
   using namespace sea::gemm;
   const int64_t m_tiles = ceil_div(rows, BM);
   const int bn = gemm_tile_n(rows, n, dev->num_sms);
+  const bool pair = bn == kPairTileN;
   const bool narrow = bn == NarrowTiles::BN;
+  // A pair CTA loads 128 rows of W (its half of the 256-column tile).
+  const uint32_t w_box_rows = pair ? PairShape::BN / 2 : static_cast<uint32_t>(bn);
   if (!encode_2d(&tx, x.ptr, d_model, rows, x.row_stride * 2, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_2d(&tw, w_qkv, d_model, n, static_cast<uint64_t>(d_model) * 2, BK, bn, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&tw, w_qkv, d_model, n, static_cast<uint64_t>(d_model) * 2, BK, w_box_rows,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_2d(&to, qkv_out.ptr, n, rows, qkv_out.row_stride * 2, EPI_COLS, 32, CU_TENSOR_MAP_SWIZZLE_64B))
     return ATTN_ERR_CUDA;
   Args a{};
@@ -441,13 +505,20 @@ attn_status attn_qkv_pack(attn_mat x, const void* w_qkv, const void* b_q, const 
   a.d_model = d_model;
   a.err = dev->err;
   a.limit_ns = sea::kDefaultTimeoutNs;
-  const int64_t tiles = m_tiles * ceil_div(n, bn);
-  const int grid = static_cast<int>(std::min<int64_t>(tiles, dev->num_sms));
-  const cudaError_t err =
-      narrow ? launch_pdl(qkv_gemm_kernel<NarrowTiles>, dim3(grid), dim3(THREADS), NarrowTiles::SMEM_BYTES, stream, tx,
-                          tw, to, a)
-             : launch_pdl(qkv_gemm_kernel<WideTiles>, dim3(grid), dim3(THREADS), WideTiles::SMEM_BYTES, stream, tx, tw,
-                          to, a);
+  cudaError_t err;
+  if (pair) {
+    const int64_t tiles = ceil_div(rows, 2 * BM) * ceil_div(n, PairShape::BN);
+    const int pairs = static_cast<int>(std::min<int64_t>(tiles, dev->num_sms / 2));
+    err = launch_pdl_cluster(qkv_gemm_pair_kernel, dim3(2 * pairs), dim3(THREADS), PairShape::SMEM_BYTES, stream, 2u,
+                             tx, tw, to, a);
+  } else {
+    const int64_t tiles = m_tiles * ceil_div(n, bn);
+    const int grid = static_cast<int>(std::min<int64_t>(tiles, dev->num_sms));
+    err = narrow ? launch_pdl(qkv_gemm_kernel<NarrowTiles>, dim3(grid), dim3(THREADS), NarrowTiles::SMEM_BYTES, stream,
+                              tx, tw, to, a)
+                 : launch_pdl(qkv_gemm_kernel<WideTiles>, dim3(grid), dim3(THREADS), WideTiles::SMEM_BYTES, stream, tx,
+                              tw, to, a);
+  }
   if (err != cudaSuccess) return ATTN_ERR_CUDA;
   return ATTN_OK;
 }
@@ -514,6 +585,14 @@ attn_status attn_cross(attn_mat q, attn_mat k_enc, attn_mat v_enc, int32_t batch
 attn_status attn_cross_static_scratch(attn_mat q, attn_mat k_enc, attn_mat v_enc, int32_t batch, int32_t t_q,
                                       int32_t t_enc, int32_t n_heads, int32_t head_dim, float scale, attn_mat out,
                                       attn_stream_t stream) {
+  attn_mask full{};
+  full.kind = ATTN_MASK_FULL;
+  // The arguments are checked before the device is queried, so an invalid
+  // call returns ATTN_ERR_INVALID without any CUDA call, as attn_cross does.
+  if (attn_status st = validate_attention(q, k_enc, v_enc, batch, t_q, t_enc, n_heads, head_dim, full, nullptr,
+                                          scale, out, nullptr, 0);
+      st != ATTN_OK)
+    return st;
   DeviceInfo* dev = nullptr;
   if (attn_status st = device_info(&dev); st != ATTN_OK) return st;
   void* scratch = nullptr;
@@ -522,8 +601,6 @@ attn_status attn_cross_static_scratch(attn_mat q, attn_mat k_enc, attn_mat v_enc
   // that needs more than kStaticScratchBytes is rejected (ATTN_ERR_INVALID)
   // before anything is launched. Every partial the combine step reads is
   // written earlier in the same call, so nothing has to be cleared.
-  attn_mask full{};
-  full.kind = ATTN_MASK_FULL;
   return launch_attention(q, k_enc, v_enc, batch, t_q, t_enc, n_heads, head_dim, full, nullptr, scale, out,
                           scratch, kStaticScratchBytes, stream);
 }

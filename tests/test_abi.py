@@ -187,8 +187,13 @@ def test_slotmask_slot_limit_is_enforced(lib):
 def test_plan_of_the_benchmarked_and_one_window_steps(lib):
     p = attn.debug_plan(8, 1500, 1500, 20, proj_rows=12000, d_model=1280)
     assert (p["q_tiles"], p["kv_splits"], p["units"], p["workspace_bytes"]) == (12, 1, 8 * 20 * 12, 0)
-    # 94 x 15 wide tiles = 9.53 waves against 94 x 20 narrow ones = 12.7: wide
-    assert p["proj_tile_n"] == 256
+    # 12000 rows: CTA-pair projection (256 x 256 tiles on two SMs) when enabled,
+    # else 94 x 15 wide tiles = 9.53 waves against 94 x 20 narrow ones = 12.7: wide
+    assert p["proj_tile_n"] in (512, 256)
+    # below 4096 rows: 32 x 15 wide tiles = 3.2 waves against 32 x 20 narrow = 4.3: wide
+    assert attn.debug_plan(1, 4000, 4000, 20, proj_rows=4000, d_model=1280)["proj_tile_n"] == 256
+    # a width that is not a multiple of 256 never takes the pair tiles
+    assert attn.debug_plan(1, 4500, 4500, 5, proj_rows=4500, d_model=320)["proj_tile_n"] in (192, 256)
     # 12 x 15 = 180 wide tiles = 2 waves, 12 x 20 = 240 narrow = 2 waves of smaller tiles: narrow
     assert attn.debug_plan(1, 1500, 1500, 20, proj_rows=1500, d_model=1280)["proj_tile_n"] == 192
 
@@ -244,3 +249,20 @@ def test_plan_rejects_invalid_requests(lib):
     assert lib.attn_debug_plan(1, 1, 1, 1, 9, 0, 148, 0, 0, ctypes.byref(info)) == attn.ATTN_ERR_INVALID
     assert lib.attn_debug_plan(1, 8, 8, 1, attn.MASK_CHUNK, 0, 148, 0, 0, ctypes.byref(info)) == attn.ATTN_ERR_INVALID
     assert lib.attn_debug_plan(1, 1, 1, 1, 0, 0, 148, 0, 0, None) == attn.ATTN_ERR_INVALID
+
+
+def call_static_scratch(lib, q=None, k=None, v=None, out=None, batch=1, t_q=80, t_enc=1500, heads=2, hd=64,
+                        scale=0.125):
+    return lib.attn_cross_static_scratch(q or m(P, 128), k or m(P2, 128), v or m(P3, 128), batch, t_q, t_enc,
+                                         heads, hd, scale, out or m(P4, 128), None)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(batch=0), dict(t_q=0), dict(t_enc=-1), dict(heads=0), dict(hd=128), dict(scale=0.0),
+    dict(q=m(0, 128)), dict(k=m(P2 + 8, 128)), dict(v=m(P3, 100)), dict(out=m(P + 64, 128)),
+])
+def test_static_scratch_rejects_invalid_arguments_before_any_cuda_call(lib, kw):
+    """The fixed-scratch cross-attention checks its arguments before it looks
+    at the device: here, with no usable device, an invalid call must still say
+    ATTN_ERR_INVALID (a device query would have failed with another status)."""
+    assert call_static_scratch(lib, **kw) == attn.ATTN_ERR_INVALID

@@ -3,15 +3,19 @@ device memory (a host that owns every device allocation through its own pool,
 or a real-time decode loop that must not allocate between frames).
 
 It runs the split-KV cross-attention with its partials in the library's fixed
-device array instead of a caller workspace. Its output must match attn_cross
-(with a caller workspace) within the parity tolerance, on two calls in a row,
-and a shape whose split needs more than the fixed 4 MiB must be refused.
-This file is named to be collected last."""
+device array instead of a caller workspace. Two calls with different queries,
+enqueued back to back on one stream with no synchronisation between them
+(the second reuses the array the first one wrote), must each match the FP64
+oracle and the workspace entry point attn_cross within the parity tolerance;
+a call after a warm-up must allocate no device memory; and a shape whose
+split needs more than the fixed 4 MiB must be refused. This file is named to
+be collected last."""
 import ctypes
 
 import numpy as np
 import pytest
 
+import oracle
 from speech_encoder_attention_b200 import attn, inputs
 from tests.gpu_util import assert_parity, to_dev, to_np64
 
@@ -24,29 +28,62 @@ def _mat(t):
     return attn.AttnMat(ctypes.c_void_p(t.data_ptr()), t.stride(0))
 
 
-def test_static_scratch_matches_workspace_entry_point_twice():
+def _verify_cross_inputs():
+    spec = inputs.VERIFY_WORKLOADS["verify"]
+    inp = inputs.make_verify_inputs(spec)
+    # a second block of queries, so the two calls' partials differ
+    q2 = inputs.random_f16(np.random.default_rng([spec.seed, 99]), inp.q.shape)
+    return spec, inp, q2
+
+
+def test_static_scratch_matches_oracle_and_workspace_entry_point_back_to_back():
     import torch
     assert torch.cuda.is_available()
     lib = attn.load_library()
-    spec = inputs.VERIFY_WORKLOADS["verify"]
-    inp = inputs.make_verify_inputs(spec)
-    q, ke, ve = (to_dev(a) for a in (inp.q, inp.k_enc, inp.v_enc))
+    spec, inp, q2_host = _verify_cross_inputs()
+    ke, ve = to_dev(inp.k_enc), to_dev(inp.v_enc)
+    qs = [to_dev(inp.q), to_dev(q2_host)]
     d = spec.d_model
     # the shape splits its key range, so the scratch is really used
     need = attn.workspace_size(1, spec.t_q, spec.t_enc, spec.n_heads, attn.MASK_FULL)
     assert 0 < need <= STATIC_SCRATCH_BYTES
 
-    want = attn.attn_cross(q, ke, ve, 1, spec.t_q, spec.t_enc, spec.n_heads)
-    torch.cuda.synchronize()
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    for call in range(2):
-        out = torch.full((spec.t_q, d), float("nan"), dtype=torch.float16, device="cuda")
+    outs = [torch.full((spec.t_q, d), float("nan"), dtype=torch.float16, device="cuda") for _ in qs]
+    for q, out in zip(qs, outs):  # no synchronisation between the two calls
+        st = lib.attn_cross_static_scratch(_mat(q), _mat(ke), _mat(ve), 1, spec.t_q, spec.t_enc, spec.n_heads,
+                                           64, 0.125, _mat(out), stream)
+        assert st == attn.ATTN_OK, attn.status_string(st)
+    torch.cuda.synchronize()
+    wants = [attn.attn_cross(q, ke, ve, 1, spec.t_q, spec.t_enc, spec.n_heads) for q in qs]
+    torch.cuda.synchronize()
+    for call, (q_host, out, want) in enumerate(zip((inp.q, q2_host), outs, wants)):
+        ref = oracle.cross_attention(q_host, inp.k_enc, inp.v_enc, spec.n_heads)
+        assert_parity(to_np64(out), ref, what=f"static scratch call {call} vs oracle")
+        assert_parity(to_np64(out), to_np64(want), what=f"static scratch call {call} vs attn_cross")
+    assert attn.debug_error_word() == (attn.ATTN_OK, 0)
+
+
+def test_static_scratch_allocates_nothing():
+    import torch
+    lib = attn.load_library()
+    spec, inp, _ = _verify_cross_inputs()
+    q, ke, ve = (to_dev(a) for a in (inp.q, inp.k_enc, inp.v_enc))
+    out = torch.empty(spec.t_q, spec.d_model, dtype=torch.float16, device="cuda")
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+    def call():
         st = lib.attn_cross_static_scratch(_mat(q), _mat(ke), _mat(ve), 1, spec.t_q, spec.t_enc, spec.n_heads,
                                            64, 0.125, _mat(out), stream)
         assert st == attn.ATTN_OK, attn.status_string(st)
         torch.cuda.synchronize()
-        assert_parity(to_np64(out), to_np64(want), what=f"static scratch call {call}")
-    assert attn.debug_error_word() == (attn.ATTN_OK, 0)
+
+    call()  # warm-up: the device set-up and lazy module loading happen here
+    free0, allocated0 = torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated()
+    for _ in range(3):
+        call()
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert torch.cuda.memory_allocated() == allocated0
 
 
 def test_static_scratch_refuses_splits_larger_than_the_array():
