@@ -137,7 +137,7 @@ REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_pow
 
 
 class ClockSampler:
-    def __init__(self, device_index: int, period_s: float = 0.02):
+    def __init__(self, device_index: int, period_s: float = 0.001):
         self.period = period_s
         self.samples = []
         self.max_mhz = None
@@ -686,6 +686,38 @@ def check_device_errors(step, where):
         raise RuntimeError(f"device error word {word:#x} after the {where}: a kernel wait timed out")
 
 
+def time_secondary(name, device, steps, warmup, ws):
+    """The bandwidth-bound verify step (token-tree SLOTMASK + cross-attention),
+    timed like the main step (L2 flushed between steps, CUDA events on the
+    launching stream, max over ranks): its step time, algorithmic bytes and
+    fraction of the HBM roofline."""
+    import torch
+    step = make_step(name, device)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    for _ in range(warmup):
+        step.run()
+    torch.cuda.synchronize()
+    nk = len(step.kernels)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(steps)]
+    for e in ev:
+        flush.zero_()
+        step.run(e)
+    torch.cuda.synchronize()
+    check_device_errors(step, f"{name} steps")
+    local_ms = sum(e[0].elapsed_time(e[nk]) for e in ev) / steps
+    ms = reduce_step_time(local_ms, device)
+    peaks, peak_kind = load_peaks()
+    total_bytes = step.total_bytes()
+    gbs = total_bytes / (ms * 1e-3) / 1e9
+    return {"workload": workload_config(step.spec)["workload"], "ms_per_step": ms,
+            "algorithmic_bytes_per_step": total_bytes, "achieved_gbs": gbs, "peak_gbs": peaks["hbm_gbs"],
+            "hbm_frac": gbs / peaks["hbm_gbs"], "peak_source": f"{peak_kind} hbm_gbs",
+            "tflops": step.total_flops() / (ms * 1e-3) / 1e12,
+            "kernels_us": {k: sum(e[i].elapsed_time(e[i + 1]) for e in ev) / steps * 1e3
+                           for i, k in enumerate(step.kernels)},
+            "launches_per_step": step.launches_per_step}
+
+
 def run_gpu(args):
     import torch
     ws, rank, local = dist_env()
@@ -749,6 +781,11 @@ def run_gpu(args):
         e2e_local = sum(a.elapsed_time(b) for a, b in eev) / n_e2e
         e2e_ms = reduce_step_time(e2e_local, device)
 
+    # the bandwidth-bound decoder step, reported beside the encoder headline
+    secondary = None
+    if isinstance(step, EncoderStep) and not args.skip_secondary:
+        secondary = time_secondary("verify", device, max(args.steps, 50), max(args.warmup, 3), ws)
+
     if ws > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -804,6 +841,7 @@ def run_gpu(args):
             "value": whole_job_rate(flops, ws, e2e_ms) / 1e12, "unit": unit,
             "h2d_bytes_per_step": step.h2d_bytes, "d2h_bytes_per_step": step.d2h_bytes,
             "ms_per_step": e2e_ms},
+        "secondary": secondary,
         "gpu_launches": step.launches_per_step * args.steps,
         "clocks": clocks.summary(),
         "kernel_source_hash": kernel_source_hash(),
@@ -825,6 +863,8 @@ def parse(argv=None):
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--skip-cpu-baseline", action="store_true")
     p.add_argument("--skip-e2e", action="store_true")
+    p.add_argument("--skip-secondary", action="store_true",
+                   help="do not time the verify step beside an encoder workload")
     args = p.parse_args(argv)
     if args.warmup < 3 and args.impl == "native":
         p.error("--warmup must be at least 3")

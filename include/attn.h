@@ -251,8 +251,9 @@ attn_status attn_debug_error_word(attn_stream_t stream, uint32_t *word_out);
  *     of whole chunks; otherwise one segment of t_q rows)
  *   kv_splits, kv_tiles_per_split: the key split (1 = none); units = work units
  *   workspace_bytes: what attn_workspace_size would report for that device
- *   proj_tile_n: the projection's output tile width for proj_rows rows of
- *     d_model (256 or 192; 0 when proj_rows or d_model is 0)
+ *   proj_tile_n: the projection's output tile for proj_rows rows of d_model:
+ *     256 or 192 (128-row tiles of that width on one SM), 512 (256 x 256
+ *     tiles on a pair of SMs), 0 when proj_rows or d_model is 0
  * Pure host arithmetic (no CUDA call). Returns ATTN_ERR_INVALID for
  * non-positive sizes or SM count, an unknown mask kind or CHUNK without a
  * positive chunk_len.

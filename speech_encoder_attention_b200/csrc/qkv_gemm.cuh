@@ -289,3 +289,236 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 }  // namespace gemm
 }  // namespace sea
+
+namespace sea {
+namespace gemm {
+
+// ---------------------------------------------------------------------------
+// CTA-pair variant: 256 x 256 output tiles computed by two SMs with
+// cta_group::2 MMAs (M = 256, N = 256, K = 16). CTA r of the pair owns tile
+// rows [128 r, 128 r + 128): it loads its 128 rows of x and its 128 rows of W
+// (the MMA splits B along N between the pair), holds its rows' accumulator in
+// its own tensor memory and writes them. Per SM this reads half the operand
+// bytes per flop of the 128 x 256 single-CTA tile. Roles as in
+// qkv_gemm_kernel; the pair leader's thread issues the MMAs, whose
+// completions are signalled to both CTAs' barriers; the peer's epilogue
+// releases an accumulator by arriving on the leader's barrier. No TMA load
+// is multicast: each CTA loads only its own halves.
+// ---------------------------------------------------------------------------
+struct PairShape {
+  static constexpr int BN = 256;  // tile columns (the pair's N)
+  static constexpr int STAGES = 6;
+  static constexpr int HALF_BYTES = 128 * BK * 2;  // one CTA's 128 rows of a 64-wide K slice
+  static constexpr int STAGE_BYTES = 2 * HALF_BYTES;  // its x half + its W half
+  static constexpr int OFF_STAGES = 0;
+  static constexpr int OFF_EPI = OFF_STAGES + STAGES * STAGE_BYTES;
+  static constexpr int OFF_BARS = OFF_EPI + EPI_BYTES;
+  // barriers: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain
+  static constexpr int NUM_BARS = 2 * STAGES + 5;
+  static constexpr int OFF_MISC = OFF_BARS + 8 * NUM_BARS;
+  static constexpr int SMEM_BYTES = 1024 + OFF_MISC + 16;
+};
+
+__global__ void __launch_bounds__(THREADS, 1)
+    qkv_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                         const __grid_constant__ CUtensorMap tm_out, const Args args) {
+  using S = PairShape;
+  constexpr int BN = S::BN;
+  constexpr int STAGES = S::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + S::OFF_BARS;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::OFF_MISC);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + S::OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0: pair leader
+  const int pair = blockIdx.x >> 1;
+  const int num_pairs = gridDim.x >> 1;
+  const int tiles_m = (args.m + 2 * BM - 1) / (2 * BM);
+  const int tiles_n = (args.n + BN - 1) / BN;
+  const int num_tiles = tiles_m * tiles_n;
+  const int kblocks = (args.k + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 8);  // the leader's: four epilogue warps of each CTA
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0u;
+    fence_barrier_init();
+    tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_w);
+    tma_prefetch_desc(&tm_out);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before either signals the other's
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  griddep_wait();
+  griddep_launch_dependents();
+  const WaitCtl wc{abort_flag, args.err, args.limit_ns};
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer (both CTAs) ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      for (int tile = pair; tile < num_tiles; tile += num_pairs) {
+        const int m0 = (tile / tiles_n) * 2 * BM + static_cast<int>(rank) * BM;
+        const int n0 = (tile % tiles_n) * BN + static_cast<int>(rank) * (BN / 2);
+        bool ok = true;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, wc)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sa = sbase + S::OFF_STAGES + stage * S::STAGE_BYTES;
+          const uint32_t leader_full = mapa_shared(full_bar(stage), 0);
+          if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * S::STAGE_BYTES);
+          tma_load_2d_pair(sa, &tm_x, leader_full, kb * BK, m0);
+          tma_load_2d_pair(sa + S::HALF_BYTES, &tm_w, leader_full, kb * BK, n0);
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+      }
+      // Let this CTA's last copies land before it can exit: once the leader's
+      // MMAs that read a stage completed, its bytes had arrived.
+      for (int i = 0; i < STAGES && i < issued; ++i) {
+        if (--stage < 0) {
+          stage = STAGES - 1;
+          phase ^= 1u;
+        }
+        mbar_wait_drain(empty_bar(stage), phase, args.limit_ns);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // ---------------- MMA issuer (pair leader) ----------------
+      constexpr uint32_t idesc = idesc_f16_f32(2 * BM, BN, 0, 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs, ++local) {
+        const int acc = local & 1;
+        const uint32_t acc_phase = (local >> 1) & 1;
+        if (!mbar_wait_cluster(tempty_bar(acc), acc_phase ^ 1u, wc)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, wc)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = sbase + S::OFF_STAGES + stage * S::STAGE_BYTES;
+          const uint32_t sb = sa + S::HALF_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = smem_desc_sw128(sa + kk * 32, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(sb + kk * 32, 16, 1024);
+            mma_f16_ss_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          mma_commit_pair(empty_bar(stage), 0x3);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (ok) mma_commit_pair(tfull_bar(acc), 0x3);
+      }
+      mma_commit_pair(drain_bar, 0x1);
+      mbar_wait_drain(drain_bar, 0, args.limit_ns);
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5, both CTAs) ----------------
+    const int quad = warp & 3;
+    const uint32_t lane_field = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t ebuf = sbase + S::OFF_EPI + (warp - 2) * 2 * EPI_BUF_BYTES;
+    uint32_t chunk_count = 0;
+    int local = 0;
+    for (int tile = pair; tile < num_tiles; tile += num_pairs, ++local) {
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      if (!mbar_wait_cluster(tfull_bar(acc), acc_phase, wc)) break;
+      tc_fence_after();
+      const int m0 = (tile / tiles_n) * 2 * BM + static_cast<int>(rank) * BM;
+      const int n0 = (tile % tiles_n) * BN;
+      const int row0 = m0 + quad * 32;
+#pragma unroll 1
+      for (int c = 0; c < BN / EPI_COLS; ++c) {
+        const int n_c = n0 + c * EPI_COLS;
+        if (n_c >= args.n) break;
+        uint32_t r[32];
+        tmem_ld32(tmem_base + acc * BN + c * EPI_COLS + lane_field, r);
+        float bias[32];
+        load_bias32(args, n_c, bias);
+        uint32_t h[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          h[i] = pack_half2(__uint_as_float(r[2 * i]) + bias[2 * i], __uint_as_float(r[2 * i + 1]) + bias[2 * i + 1]);
+        const uint32_t buf = ebuf + (chunk_count & 1u) * EPI_BUF_BYTES;
+        if (lane == 0) bulk_wait_group_read<1>();
+        __syncwarp();
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const uint32_t addr = buf + lane * 64 + ((v ^ ((lane >> 1) & 3)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(h[4 * v]), "r"(h[4 * v + 1]),
+                       "r"(h[4 * v + 2]), "r"(h[4 * v + 3])
+                       : "memory");
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && row0 < args.m) {
+          tma_store_2d(&tm_out, buf, n_c, row0);
+          bulk_commit_group();
+        }
+        ++chunk_count;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (rank == 0)
+          mbar_arrive(tempty_bar(acc));
+        else
+          mbar_arrive_remote(mapa_shared(tempty_bar(acc), 0));
+      }
+    }
+    if (lane == 0) bulk_wait_group_all();
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // neither CTA frees tensor memory the pair's MMAs may still use
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace gemm
+}  // namespace sea

@@ -119,6 +119,32 @@ def test_qkv_projection_shapes(rows, d):
     assert_parity(to_np64(got), oracle.qkv_projection(x, w, bq, bv), what=f"qkv {rows}x{d}")
 
 
+@pytest.mark.parametrize("rows,d", [(4096, 256), (4097, 512), (5000, 1280), (8191, 1024), (4500, 320)])
+def test_qkv_projection_on_cta_pairs(rows, d):
+    """Row counts that take the CTA-pair projection (256 x 256 tiles over two
+    SMs): whole and ragged pair tiles, a last tile whose second CTA has no
+    row, and a width (3 x 320) that is not a multiple of 256, which falls
+    back to single-CTA tiles."""
+    torch = torch_mod()
+    rng = np.random.default_rng(rows + d)
+    x = inputs.random_f16(rng, (rows, d))
+    w = inputs.random_f16(rng, (3 * d, d), 0.02)
+    bq = inputs.random_f16(rng, (d,), 0.01)
+    bv = inputs.random_f16(rng, (d,), 0.01)
+    if rows == 4097:
+        bq = bv = None
+    big = torch.full((rows, 3 * d + 32), 7.0, dtype=torch.float16, device="cuda")
+    out = big[:, :3 * d]
+    attn.attn_qkv_pack(to_dev(x), to_dev(w), None if bq is None else to_dev(bq), None if bv is None else to_dev(bv),
+                       out=out)
+    torch.cuda.synchronize()
+    zero = np.zeros(d, dtype=np.float16)
+    want = oracle.qkv_projection(x, w, zero if bq is None else bq, zero if bv is None else bv)
+    assert_parity(to_np64(out), want, what=f"qkv pairs {rows}x{d}")
+    assert torch.all(big[:, 3 * d:] == 7.0), "wrote outside the output view"
+    check_error_word()
+
+
 def test_qkv_projection_without_bias_and_padded_output():
     torch = torch_mod()
     rng = np.random.default_rng(5)
@@ -248,6 +274,34 @@ def test_large_logits_do_not_overflow():
     ref = oracle.attention(q, k, v, 2, oracle.allowed_full(300, 300))
     # v has std 4 here, so scale the absolute bound with it
     assert_parity(to_np64(got), ref, abs_tol=4 * 5e-3, what="large logits")
+
+
+@pytest.mark.parametrize("order", ["growing", "shrinking", "mixed"])
+def test_row_max_jumps_between_key_tiles(order):
+    """Key tiles whose logits jump by far more than the softmax's exponent
+    headroom from one tile to the next (the range kernel computes a tile's
+    exponentials against the reference of earlier tiles and must redo the tile
+    and rescale O and the row sums when a row's max outgrows it): keys
+    [512, 1024) are scaled up 6x, so their logits reach ~20 natural units
+    above those of the first tiles. "mixed" shrinks every other query row
+    twenty-fold, so those rows never outgrow their reference while their
+    neighbours in the same warp do."""
+    torch = torch_mod()
+    rng = np.random.default_rng({"growing": 31, "shrinking": 32, "mixed": 33}[order])
+    t, heads = 1300, 2
+    q = rng.standard_normal((t, heads * 64))
+    k = rng.standard_normal((t, heads * 64))
+    v = rng.standard_normal((t, heads * 64))
+    big = slice(512, 1024) if order != "shrinking" else slice(0, 512)
+    k[big] *= 6.0
+    if order == "mixed":
+        q[1::2] *= 0.05
+    q, k, v = (a.astype(np.float16) for a in (q, k, v))
+    got = attn.attn_forward(to_dev(q), to_dev(k), to_dev(v), 1, t, t, heads)
+    torch.cuda.synchronize()
+    check_error_word()
+    ref = oracle.attention(q, k, v, heads, oracle.allowed_full(t, t))
+    assert_parity(to_np64(got), ref, what=f"row max jumps ({order})")
 
 
 def test_output_view_padding_untouched_and_strided_inputs():
