@@ -262,7 +262,7 @@ constexpr bool kRangeKernelV2 = SEA_RANGE_KERNEL_V2 != 0;
 // Row counts from which the projection runs on CTA pairs (256 x 256 tiles,
 // cta_group::2): large enough that the pair tiles fill the GPU.
 #ifndef SEA_PAIR_MIN_ROWS
-#define SEA_PAIR_MIN_ROWS (1 << 30)
+#define SEA_PAIR_MIN_ROWS 4096
 #endif
 constexpr int64_t kPairMinRows = SEA_PAIR_MIN_ROWS;
 constexpr int kPairTileN = 512;  // plan code for the pair kernel (tile 256 rows x 256 columns)

@@ -107,14 +107,17 @@ struct Cfg {
 };
 
 // Lazy rescaling: the exponent reference m only moves when a row's max grows
-// by more than this (log2 units), so p <= 2^8 fits fp16 and O is rescaled rarely.
-constexpr float RESCALE_THRESHOLD = 8.0f;
+// by more than this (log2 units), so p <= 2^15 fits fp16 and O is rescaled rarely.
+constexpr float RESCALE_LIMIT = 15.0f;
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Bit k set: pair k (mod 8) of every 16 keys takes the FMA-pipe exp2 instead
+// Bit k set: pair k of every 16 keys takes the FMA-pipe exp2 instead
 // of MUFU ex2. Measured on B200 the extra instructions cost more than the
 // MUFU relief buys in this kernel, so no pair is moved.
-constexpr uint32_t POLY_PAIRS = 0x00u;
+#ifndef SEA_POLY_PAIRS
+#define SEA_POLY_PAIRS 0x00u
+#endif
+constexpr uint32_t POLY_PAIRS = SEA_POLY_PAIRS;
 
 struct TileGeom {
   int q0;     // first query row (sequence-local)
@@ -479,7 +482,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, Cfg::MIN_BLOCKS)
       // Allowed key range of this row for the range family (sequence-local indices).
       int lo_i = 0, hi_i = 0;
       if (!use_flags && row_ok) row_keys<EXT>(p, seq_len<EXT>(p, U.b), row_glob, lo_i, hi_i);
-      float m_run = -INFINITY;  // exponent reference (log2 units), lags the true max by < 8
+      float m_run = -INFINITY;  // exponent reference (log2 units), lags the true max by <= 15
       float l_run = 0.f;
       int t_unit = 0;  // tiles of this unit done
       for (int j = U.j_begin; j < U.j_end; ++j) {
@@ -522,65 +525,69 @@ __global__ void __launch_bounds__(Cfg::THREADS, Cfg::MIN_BLOCKS)
               if (e < a || e >= bnd) s[e] = -INFINITY;
           }
         }
-        // row max: eight independent chains of 3-input max, then a short tree
-        float mx;
-        {
-          float mx8[8];
+        // The tile's row max: eight independent chains of 3-input max.
+        auto row_max = [&]() -> float {
+          float mx4[4];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) mx8[i] = s[i];
+          for (int i = 0; i < 4; ++i) mx4[i] = fmaxf(s[i], s[124 + i]);
 #pragma unroll
-          for (int e = 8; e < 128; e += 16) {
+          for (int e = 4; e < 124; e += 8) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) mx8[i] = fmax3(mx8[i], s[e + i], s[e + 8 + i]);
+            for (int i = 0; i < 4; ++i) mx4[i] = fmax3(mx4[i], s[e + i], s[e + 4 + i]);
           }
-          mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
-        }
+          return fmaxf(fmax3(mx4[0], mx4[1], mx4[2]), mx4[3]);
+        };
+        // p = 2^(s*scale*log2e - m), summed in fp32 and written to P as fp16
+        // pairs, 32 keys at a time. MUFU ex2 serves 16 lanes per clock per SM;
+        // pairs picked by POLY_PAIRS take the FMA-pipe exp2 instead.
+        auto exp_tile = [&](float m_use) -> float {
+          const uint64_t sl2x2 = f2_pack(sl2, sl2);
+          const uint64_t negm2 = f2_pack(-m_use, -m_use);
+          uint64_t acc2[2] = {0ull, 0ull};
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint32_t pk[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              float x0, x1, p0, p1;
+              f2_unpack(f2_fma(f2_pack(s[16 * c + 2 * i], s[16 * c + 2 * i + 1]), sl2x2, negm2), x0, x1);
+              if ((POLY_PAIRS >> i) & 1) {
+                exp2_poly_x2(x0, x1, p0, p1);
+              } else {
+                p0 = ex2_approx(x0);
+                p1 = ex2_approx(x1);
+              }
+              acc2[i & 1] = f2_add(acc2[i & 1], f2_pack(p0, p1));
+              pk[i] = pack_half2(p0, p1);
+            }
+            tmem_st8_async(p_tmem + c * 8, pk);
+          }
+          tmem_wait_st();
+          float sum0, sum1;
+          f2_unpack(f2_add(acc2[0], acc2[1]), sum0, sum1);
+          return sum0 + sum1;
+        };
+        // Move the exponent reference only when the row max grew by more than
+        // RESCALE_LIMIT since it was set (lazy rescaling).
+        const float mx = row_max();
         const float mx_l2 = mx * sl2;
-        // Move the reference only when the max grew by more than the threshold.
-        const bool grow = mx_l2 > m_run + RESCALE_THRESHOLD;
+        const bool grow = mx_l2 > m_run + RESCALE_LIMIT;
         const float m_new = grow ? mx_l2 : m_run;
-        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-        const float alpha = grow ? ex2_approx(m_run - m_use) : 1.f;
+        const float alpha = grow ? ex2_approx(m_run - m_new) : 1.f;  // 0 while the reference was -inf
+        const bool first = t_unit == 0;
         // P and O are still read by this unit's previous PV until it completes
         // (for a unit's first tile the previous unit's epilogue waited already).
-        if (t_unit > 0) {
+        if (!first) {
           if (!mbar_wait(o_done, (it - 1) & 1, wc)) {
             ok = false;
             break;
           }
           tc_fence_after();
         }
-        // p = 2^(s*scale*log2e - m), summed in fp32 and written to P as fp16
-        // pairs, 32 keys at a time. MUFU ex2 serves 16 lanes per clock per SM;
-        // pairs picked by POLY_PAIRS take the FMA-pipe exp2 instead.
-        const uint64_t sl2x2 = f2_pack(sl2, sl2);
-        const uint64_t negm2 = f2_pack(-m_use, -m_use);
-        uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float x0, x1, p0, p1;
-            f2_unpack(f2_fma(f2_pack(s[32 * c + 2 * i], s[32 * c + 2 * i + 1]), sl2x2, negm2), x0, x1);
-            if ((POLY_PAIRS >> (i & 7)) & 1) {
-              exp2_poly_x2(x0, x1, p0, p1);
-            } else {
-              p0 = ex2_approx(x0);
-              p1 = ex2_approx(x1);
-            }
-            acc2[i & 3] = f2_add(acc2[i & 3], f2_pack(p0, p1));
-            pk[i] = pack_half2(p0, p1);
-          }
-          tmem_st16_async(p_tmem + c * 16, pk);
-        }
-        tmem_wait_st();
-        float sum0, sum1;
-        f2_unpack(f2_add(f2_add(acc2[0], acc2[1]), f2_add(acc2[2], acc2[3])), sum0, sum1);
-        l_run = l_run * alpha + (sum0 + sum1);
+        l_run = l_run * alpha + exp_tile(m_new == -INFINITY ? 0.f : m_new);
         // O holds this unit's earlier PVs (o_done above); this tile's PV is
         // only issued after p_full, so rescale it now.
-        if (t_unit > 0 && __any_sync(0xffffffffu, grow)) {
+        if (!first && __any_sync(0xffffffffu, grow)) {
 #pragma unroll 1
           for (int c = 0; c < 2; ++c) {
             uint32_t r[32];

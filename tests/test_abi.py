@@ -187,9 +187,8 @@ def test_slotmask_slot_limit_is_enforced(lib):
 def test_plan_of_the_benchmarked_and_one_window_steps(lib):
     p = attn.debug_plan(8, 1500, 1500, 20, proj_rows=12000, d_model=1280)
     assert (p["q_tiles"], p["kv_splits"], p["units"], p["workspace_bytes"]) == (12, 1, 8 * 20 * 12, 0)
-    # 12000 rows: CTA-pair projection (256 x 256 tiles on two SMs) when enabled,
-    # else 94 x 15 wide tiles = 9.53 waves against 94 x 20 narrow ones = 12.7: wide
-    assert p["proj_tile_n"] in (512, 256)
+    # 12000 rows take the CTA-pair projection (256 x 256 tiles on two SMs)
+    assert p["proj_tile_n"] == 512
     # below 4096 rows: 32 x 15 wide tiles = 3.2 waves against 32 x 20 narrow = 4.3: wide
     assert attn.debug_plan(1, 4000, 4000, 20, proj_rows=4000, d_model=1280)["proj_tile_n"] == 256
     # a width that is not a multiple of 256 never takes the pair tiles
