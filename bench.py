@@ -296,6 +296,37 @@ class EncoderStep:
         return {"frames": self.spec.batch * self.spec.t}
 
 
+class GraphedCalls:
+    """A step's library calls, each captured once in its own CUDA graph and
+    replayed every step. The decode-side calls take microseconds on the GPU,
+    less than the host spends per call (argument marshalling, three tensor-map
+    encodings, the launch); launched directly, that host time would show up as
+    device idle time between the timing events. Replaying a graph per call
+    leaves one event between consecutive calls, so each call is still timed
+    on its own."""
+
+    def __init__(self, calls):
+        import torch
+        for fn in calls:  # warm-up: per-device set-up and lazy module loading
+            fn()
+        torch.cuda.synchronize()
+        self.graphs = []
+        for fn in calls:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fn()
+            self.graphs.append(g)
+        torch.cuda.synchronize()
+
+    def run(self, events=None):
+        for i, g in enumerate(self.graphs):
+            if events:
+                events[i].record()
+            g.replay()
+        if events:
+            events[len(self.graphs)].record()
+
+
 class VerifyStep:
     """Token-tree self-attention (SLOTMASK) plus cross-attention of the same block."""
 
@@ -326,19 +357,21 @@ class VerifyStep:
             "slotmask_attn": b * d * (spec.t_q + 2 * spec.slots + spec.t_q) + 4 * inp.bits.size,
             "cross_attn": b * d * (spec.t_q + 2 * spec.t_enc + spec.t_q),
         }
-        self.launches_per_step = 4  # two attention kernels, each followed by its split combine
+        # two attention kernels, each followed by a combine kernel unless its
+        # key split merges inside a thread-block cluster
+        sms = torch.cuda.get_device_properties(device).multi_processor_count
+        plans = (attn.debug_plan(1, spec.t_q, spec.slots, spec.n_heads, attn.MASK_SLOTMASK, num_sms=sms),
+                 attn.debug_plan(1, spec.t_q, spec.t_enc, spec.n_heads, attn.MASK_FULL, num_sms=sms))
+        self.launches_per_step = sum(1 + (pl["kv_splits"] > 1 and not pl["cluster_merge"]) for pl in plans)
+        a, s = self.attn, self.spec
+        self.graphed = GraphedCalls([
+            lambda: a.attn_forward(self.q, self.kc, self.vc, 1, s.t_q, s.slots, s.n_heads,
+                                   mask_kind=a.MASK_SLOTMASK, bits=self.bits, out=self.o_self, workspace=self.ws),
+            lambda: a.attn_cross(self.q, self.ke, self.ve, 1, s.t_q, s.t_enc, s.n_heads, out=self.o_cross,
+                                 workspace=self.ws)])
 
     def run(self, events=None):
-        a, s = self.attn, self.spec
-        if events:
-            events[0].record()
-        a.attn_forward(self.q, self.kc, self.vc, 1, s.t_q, s.slots, s.n_heads, mask_kind=a.MASK_SLOTMASK,
-                       bits=self.bits, out=self.o_self, workspace=self.ws)
-        if events:
-            events[1].record()
-        a.attn_cross(self.q, self.ke, self.ve, 1, s.t_q, s.t_enc, s.n_heads, out=self.o_cross, workspace=self.ws)
-        if events:
-            events[2].record()
+        self.graphed.run(events)
 
     def run_e2e(self, events=None):
         if events:
@@ -394,14 +427,13 @@ class DrafterStep:
         self.bytes = {"drafter_attn": 2 * d * spec.beams * (2 * spec.t_q + 2 * spec.t_kv) + 4 * spec.n_heads}
         self.launches_per_step = self.split_launches
 
-    def run(self, events=None):
         a, s = self.attn, self.spec
-        if events:
-            events[0].record()
-        a.attn_forward(self.q, self.k, self.v, s.beams, s.t_q, s.t_kv, s.n_heads, causal=s.causal,
-                       sinks=self.sinks, out=self.out, workspace=self.ws)
-        if events:
-            events[1].record()
+        self.graphed = GraphedCalls([
+            lambda: a.attn_forward(self.q, self.k, self.v, s.beams, s.t_q, s.t_kv, s.n_heads, causal=s.causal,
+                                   sinks=self.sinks, out=self.out, workspace=self.ws)])
+
+    def run(self, events=None):
+        self.graphed.run(events)
 
     def run_e2e(self, events=None):
         if events:
@@ -450,12 +482,11 @@ class Q8Step:
         self.bytes = {"q8_proj": inp.w_blocks.nbytes + 2 * spec.rows * d + 2 * spec.rows * 3 * d}
         self.launches_per_step = 1
 
+        self.graphed = GraphedCalls([
+            lambda: self.attn.attn_qkv_pack_q8_0(self.x, self.w, self.bq, self.bv, out=self.out)])
+
     def run(self, events=None):
-        if events:
-            events[0].record()
-        self.attn.attn_qkv_pack_q8_0(self.x, self.w, self.bq, self.bv, out=self.out)
-        if events:
-            events[1].record()
+        self.graphed.run(events)
 
     def run_e2e(self, events=None):
         if events:

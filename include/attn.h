@@ -64,6 +64,12 @@ typedef enum {
   ATTN_ERR_TIMEOUT = 4      /* a kernel's bounded wait expired (see attn_debug_error_word) */
 } attn_status;
 
+/* attn_mask.flags bits */
+enum {
+  ATTN_FLAG_NO_SPLIT = 1  /* never split the key range over several CTAs (one
+                             CTA per query tile: a fixed summation order) */
+};
+
 typedef enum {
   ATTN_MASK_FULL = 0,     /* every key: the bidirectional encoder window */
   ATTN_MASK_CHUNK = 1,    /* keys in the query's chunk of chunk_len frames */
@@ -95,7 +101,7 @@ typedef struct {
   int32_t window;          /* BAND: >= 1 (values above t_q + t_kv act as t_q + t_kv);
                               0 for every other kind */
   int32_t causal;          /* 0 or 1; 1 also requires j <= p_i (range family only) */
-  int32_t reserved;        /* must be 0 */
+  int32_t flags;           /* 0 or ATTN_FLAG_NO_SPLIT */
   const int32_t *q_lens;   /* range family, optional: device pointer, [batch] int32,
                               valid query rows per sequence; NULL = t_q. Values are
                               clamped to [0, t_q] on the device. 4-byte aligned. */
@@ -162,11 +168,18 @@ attn_status attn_qkv_pack_q8_0(attn_mat x, const void *w_q8_0, const void *b_q, 
  * head_dim must be 64. Scores, the running max and sum and the output
  * accumulate in fp32; the softmax weights are rounded to fp16 for the value
  * product; the output is rounded once to fp16.
+ * Short query blocks split their key range over several CTAs. A split into
+ * at most 8 parts is merged inside a thread-block cluster (the parts combine
+ * through distributed shared memory) and needs no workspace; a longer split
+ * keeps its partials in the workspace and merges them in a second kernel.
+ * mask.flags = ATTN_FLAG_NO_SPLIT turns every split off (one CTA walks each
+ * query tile's whole key range, so the summation order does not depend on
+ * the SM count); the result agrees within rounding.
  * workspace: device scratch of at least attn_workspace_size(...) bytes, 16-byte
- * aligned, used to split long key ranges of short query blocks over more SMs.
- * Passing workspace == NULL with workspace_bytes == 0 disables the split (the
- * result is the same, only the schedule differs); a non-NULL workspace smaller
- * than required returns ATTN_ERR_INVALID.
+ * aligned (0 bytes, NULL allowed, when no workspace split is planned).
+ * Passing workspace == NULL with workspace_bytes == 0 where a workspace split
+ * is planned runs that shape unsplit; a non-NULL workspace smaller than
+ * required returns ATTN_ERR_INVALID.
  */
 attn_status attn_forward(attn_mat q, attn_mat k, attn_mat v, int32_t batch, int32_t t_q,
                          int32_t t_kv, int32_t n_heads, int32_t head_dim, attn_mask mask,
@@ -209,14 +222,15 @@ attn_status attn_cross(attn_mat q, attn_mat k_enc, attn_mat v_enc, int32_t batch
  * speech plugin whose host owns every device allocation through its own
  * pool, or a real-time decode loop that must not allocate between frames.
  * Same arguments, result and error behaviour as attn_cross, without the
- * workspace: the split-KV partials live in a fixed 4 MiB array in the
- * library's device memory (one per device, held until the process exits).
+ * workspace: the partials of a split that needs a workspace (more than 8
+ * key splits) live in a fixed 4 MiB array in the library's device memory
+ * (one per device, held until the process exits).
  *   - The first call on a device looks up that array's address; make it
  *     before any stream capture on that device.
  *   - A shape whose split needs more than 4 MiB (splits x batch x n_heads x
  *     t_q x 264 bytes; splits only happen when batch*n_heads*ceil(t_q/128)
- *     is at most half the SM count) returns ATTN_ERR_INVALID and launches
- *     nothing.
+ *     is at most half the SM count, and need the array only beyond 8 splits)
+ *     returns ATTN_ERR_INVALID and launches nothing.
  *   - Every call uses the same array. Calls whose kernels may overlap on the
  *     GPU (different streams, or other devices' threads with this device
  *     current) race on it: order them on one stream.
@@ -228,7 +242,8 @@ attn_status attn_cross_static_scratch(attn_mat q, attn_mat k_enc, attn_mat v_enc
 
 /*
  * attn_workspace_size -- bytes of workspace attn_forward / attn_cross use for
- * these sizes on the current device (0 when no split is planned).
+ * these sizes on the current device (0 when no split, or a split merged in a
+ * cluster, is planned).
  */
 size_t attn_workspace_size(int32_t batch, int32_t t_q, int32_t t_kv, int32_t n_heads,
                            int32_t head_dim, int32_t mask_kind);
@@ -251,6 +266,7 @@ attn_status attn_debug_error_word(attn_stream_t stream, uint32_t *word_out);
  *     of whole chunks; otherwise one segment of t_q rows)
  *   kv_splits, kv_tiles_per_split: the key split (1 = none); units = work units
  *   workspace_bytes: what attn_workspace_size would report for that device
+ *   cluster_merge: 1 when the split parts merge inside a cluster (no workspace)
  *   proj_tile_n: the projection's output tile for proj_rows rows of d_model:
  *     256 or 192 (128-row tiles of that width on one SM), 512 (256 x 256
  *     tiles on a pair of SMs), 0 when proj_rows or d_model is 0
@@ -264,6 +280,7 @@ typedef struct {
   int32_t proj_tile_n;
   int64_t units;
   size_t workspace_bytes;
+  int32_t cluster_merge;
 } attn_plan_info;
 
 attn_status attn_debug_plan(int32_t batch, int32_t t_q, int32_t t_kv, int32_t n_heads, int32_t mask_kind,

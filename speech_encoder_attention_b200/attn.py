@@ -9,6 +9,7 @@ The function names match the C entry points:
     attn_qkv_pack(x, w_qkv, b_q, b_v, out=None)        -> qkv
     attn_qkv_pack_q8_0(x, w_q8_0, b_q, b_v, out=None)  -> qkv
     attn_forward(q, k, v, batch, t_q, t_kv, n_heads, mask=..., out=None) -> out
+      (split=False sets ATTN_FLAG_NO_SPLIT)
     attn_forward with sinks=...                          -> attn_forward_sinks
     attn_cross(q, k_enc, v_enc, batch, t_q, t_enc, n_heads, out=None)   -> out
 """
@@ -27,6 +28,8 @@ ATTN_ERR_INVALID = 1
 ATTN_ERR_UNSUPPORTED = 2
 ATTN_ERR_CUDA = 3
 ATTN_ERR_TIMEOUT = 4
+
+ATTN_FLAG_NO_SPLIT = 1
 
 MASK_FULL = 0
 MASK_CHUNK = 1
@@ -49,7 +52,7 @@ class AttnMask(ctypes.Structure):
         ("words_per_row", ctypes.c_int32),
         ("window", ctypes.c_int32),
         ("causal", ctypes.c_int32),
-        ("reserved", ctypes.c_int32),
+        ("flags", ctypes.c_int32),
         ("q_lens", ctypes.c_void_p),
         ("kv_lens", ctypes.c_void_p),
     ]
@@ -65,6 +68,7 @@ class AttnPlanInfo(ctypes.Structure):
         ("proj_tile_n", ctypes.c_int32),
         ("units", ctypes.c_int64),
         ("workspace_bytes", ctypes.c_size_t),
+        ("cluster_merge", ctypes.c_int32),
     ]
 
 
@@ -213,7 +217,7 @@ def make_mask(kind: int = MASK_FULL, chunk_len: int = 0, bits=None, window: int 
     m.chunk_len = chunk_len
     m.window = window
     m.causal = 1 if causal else 0
-    m.reserved = 0
+    m.flags = 0
     m.q_lens = _lens_ptr(q_lens)
     m.kv_lens = _lens_ptr(kv_lens)
     if kind == MASK_SLOTMASK:
@@ -253,6 +257,8 @@ def attn_forward(q, k, v, batch, t_q, t_kv, n_heads, mask_kind=MASK_FULL, chunk_
     import torch
     lib = load_library()
     mask = make_mask(mask_kind, chunk_len, bits, window, causal, q_lens, kv_lens)
+    if not split:
+        mask.flags = ATTN_FLAG_NO_SPLIT
     if out is None:
         out = torch.empty(batch * t_q, n_heads * HEAD_DIM, dtype=torch.float16, device=q.device)
     need = workspace_size(batch, t_q, t_kv, n_heads, mask_kind) if split else 0
@@ -272,7 +278,10 @@ def attn_forward(q, k, v, batch, t_q, t_kv, n_heads, mask_kind=MASK_FULL, chunk_
 
 def attn_cross(q, k_enc, v_enc, batch, t_q, t_enc, n_heads, scale=DEFAULT_SCALE, out=None,
                workspace=None, split=True, stream=None):
-    """Decoder queries against every encoder frame (FULL, t_q != t_enc allowed)."""
+    """Decoder queries against every encoder frame (FULL, t_q != t_enc allowed).
+    split=False passes no workspace: a split that needs one does not happen, a
+    split merged inside a cluster still does (attn_cross takes no flags; use
+    attn_forward with split=False for a fixed summation order)."""
     import torch
     lib = load_library()
     if out is None:

@@ -178,8 +178,14 @@ struct FaPlan {
   int seg_len, tiles_per_seg, q_tiles;
   int n_kv_max;
   int kv_splits, kv_tiles_per_split;
+  bool merge;  // splits merged inside a thread-block cluster (no workspace)
   size_t ws_bytes;
 };
+
+// Splits up to this many are merged through distributed shared memory in a
+// cluster of that many CTAs (the portable cluster size); more need the
+// workspace and the combine kernel.
+constexpr int kMaxClusterSplits = 8;
 
 int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
 
@@ -211,8 +217,11 @@ FaPlan plan_forward(int batch, int t_q, int t_kv, int n_heads, int mask_kind, in
     if (splits > 1) {
       pl.kv_splits = splits;
       pl.kv_tiles_per_split = per;
-      const size_t rows = static_cast<size_t>(splits) * batch * n_heads * t_q;
-      pl.ws_bytes = rows * sea::fa::DH * sizeof(float) + rows * 2 * sizeof(float);
+      pl.merge = splits <= kMaxClusterSplits;
+      if (!pl.merge) {
+        const size_t rows = static_cast<size_t>(splits) * batch * n_heads * t_q;
+        pl.ws_bytes = rows * sea::fa::DH * sizeof(float) + rows * 2 * sizeof(float);
+      }
     }
   }
   return pl;
@@ -299,7 +308,7 @@ attn_status validate_attention(attn_mat q, attn_mat k, attn_mat v, int32_t batch
   if (!valid_mat(q, cols) || !valid_mat(k, cols) || !valid_mat(v, cols) || !valid_mat(out, cols))
     return ATTN_ERR_INVALID;
   auto misaligned4 = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 3u) != 0; };
-  if (mask.reserved != 0) return ATTN_ERR_INVALID;
+  if ((mask.flags & ~ATTN_FLAG_NO_SPLIT) != 0) return ATTN_ERR_INVALID;
   if (mask.causal != 0 && mask.causal != 1) return ATTN_ERR_INVALID;
   if (mask.kind != ATTN_MASK_BAND && mask.window != 0) return ATTN_ERR_INVALID;
   if (misaligned4(mask.q_lens) || misaligned4(mask.kv_lens) || misaligned4(sinks)) return ATTN_ERR_INVALID;
@@ -339,7 +348,18 @@ attn_status launch_attention(attn_mat q, attn_mat k, attn_mat v, int32_t batch, 
   if (attn_status st = device_info(&dev); st != ATTN_OK) return st;
 
   FaPlan pl = plan_forward(batch, t_q, t_kv, n_heads, mask.kind, mask.chunk_len, dev->num_sms);
-  if (pl.kv_splits > 1) {
+  if (mask.flags & ATTN_FLAG_NO_SPLIT) {
+    pl.kv_splits = 1;
+    pl.kv_tiles_per_split = pl.n_kv_max;
+    pl.merge = false;
+    pl.ws_bytes = 0;
+  }
+  if (pl.merge && mask.kind != ATTN_MASK_SLOTMASK && kRangeKernelV2) {
+    pl.merge = false;  // that kernel writes its partials to the workspace only
+    const size_t rows = static_cast<size_t>(pl.kv_splits) * batch * n_heads * t_q;
+    pl.ws_bytes = rows * sea::fa::DH * sizeof(float) + rows * 2 * sizeof(float);
+  }
+  if (pl.kv_splits > 1 && !pl.merge) {
     if (workspace == nullptr) {
       pl.kv_splits = 1;  // caller opted out of the split: same result, one CTA per key range
       pl.kv_tiles_per_split = pl.n_kv_max;
@@ -383,8 +403,9 @@ attn_status launch_attention(attn_mat q, attn_mat k, attn_mat v, int32_t batch, 
   p.out_stride = out.row_stride;
   float* ws = static_cast<float*>(workspace);
   const size_t ws_rows = static_cast<size_t>(pl.kv_splits) * batch * n_heads * t_q;
-  p.ws_o = pl.kv_splits > 1 ? ws : nullptr;
-  p.ws_ml = pl.kv_splits > 1 ? ws + ws_rows * sea::fa::DH : nullptr;
+  p.ws_o = pl.kv_splits > 1 && !pl.merge ? ws : nullptr;
+  p.ws_ml = pl.kv_splits > 1 && !pl.merge ? ws + ws_rows * sea::fa::DH : nullptr;
+  p.merge = pl.merge ? 1 : 0;
   p.err = dev->err;
   p.limit_ns = sea::kDefaultTimeoutNs;
 
@@ -398,12 +419,14 @@ attn_status launch_attention(attn_mat q, attn_mat k, attn_mat v, int32_t batch, 
   const int threads = sea::fa::Cfg::THREADS;
   const int smem = sea::fa::Cfg::SMEM_BYTES;
   cudaError_t err;
-  if (slot) {
-    // One unit per CTA (its tile flags need a pass over every row's words).
-    if (ext)
-      err = launch_pdl(sea::fa::flash_attn_kernel<true, true>, dim3(p.units), dim3(threads), smem, stream, tq, tk, tv, p);
-    else
-      err = launch_pdl(sea::fa::flash_attn_kernel<true, false>, dim3(p.units), dim3(threads), smem, stream, tq, tk, tv, p);
+  // A merged split runs one unit per CTA, the splits of a query tile (units
+  // next to each other) forming one cluster.
+  const unsigned cluster = pl.merge ? static_cast<unsigned>(pl.kv_splits) : 1u;
+  if (slot || pl.merge) {
+    // One unit per CTA (SLOTMASK: its tile flags need a pass over every row's words).
+    auto kern = slot ? (ext ? sea::fa::flash_attn_kernel<true, true> : sea::fa::flash_attn_kernel<true, false>)
+                     : (ext ? sea::fa::flash_attn_kernel<false, true> : sea::fa::flash_attn_kernel<false, false>);
+    err = launch_pdl_cluster(kern, dim3(p.units), dim3(threads), smem, stream, cluster, tq, tk, tv, p);
   } else if (kRangeKernelV2) {
     // Persistent: one CTA per SM walks the units.
     using FR = sea::fr::Cfg;
@@ -423,7 +446,7 @@ attn_status launch_attention(attn_mat q, attn_mat k, attn_mat v, int32_t batch, 
       err = launch_pdl(sea::fa::flash_attn_kernel<false, false>, dim3(grid), dim3(threads), smem, stream, tq, tk, tv, p);
   }
   if (err != cudaSuccess) return ATTN_ERR_CUDA;
-  if (pl.kv_splits > 1) {
+  if (pl.kv_splits > 1 && !pl.merge) {
     const int64_t rows = static_cast<int64_t>(batch) * n_heads * t_q;
     if (launch_pdl(sea::fa::combine_kernel, dim3(ceil_div(rows, 8)), dim3(256), 0, stream,
                    static_cast<const float*>(p.ws_o), static_cast<const float*>(p.ws_ml), pl.kv_splits, batch,
@@ -652,6 +675,7 @@ attn_status attn_debug_plan(int32_t batch, int32_t t_q, int32_t t_kv, int32_t n_
   out->kv_tiles_per_split = pl.kv_tiles_per_split;
   out->units = static_cast<int64_t>(batch) * n_heads * pl.q_tiles * pl.kv_splits;
   out->workspace_bytes = pl.ws_bytes;
+  out->cluster_merge = pl.merge ? 1 : 0;
   out->proj_tile_n = (proj_rows > 0 && d_model > 0) ? gemm_tile_n(proj_rows, 3 * static_cast<int64_t>(d_model), num_sms)
                                                     : 0;
   return ATTN_OK;

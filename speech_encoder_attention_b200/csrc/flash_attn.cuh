@@ -78,6 +78,10 @@ struct Params {
   int64_t out_stride;
   float* ws_o;   // [splits][batch][heads][t_q][64] unnormalised partial O
   float* ws_ml;  // [splits][batch][heads][t_q][2]  (m in log2 units, l)
+  // Split partials merged inside a thread-block cluster (one CTA per split,
+  // the cluster = one query tile's splits) instead of through ws_o / ws_ml
+  // and the combine kernel.
+  int merge;
   uint32_t* err;
   uint64_t limit_ns;
 };
@@ -302,6 +306,11 @@ __global__ void __launch_bounds__(Cfg::THREADS, Cfg::MIN_BLOCKS)
   griddep_launch_dependents();
   const WaitCtl wc{abort_flag, p.err, p.limit_ns};
   const int srow = (warp & 3) * 32 + lane;  // softmax: row within the tile == TMEM lane
+  // Cluster merge: this CTA's partial O (128 x 64 fp32) and (m, l) per row,
+  // in the K/V stages, which no copy or MMA uses once the unit's last P V
+  // has completed.
+  float* merge_o = reinterpret_cast<float*>(smem + C::OFF_K);
+  float2* merge_ml = reinterpret_cast<float2*>(smem + C::OFF_K + BQ * DH * 4);
 
   // SLOTMASK: mark the key tiles any row of this CTA's (single) unit may see.
   if constexpr (use_flags) {
@@ -464,10 +473,11 @@ __global__ void __launch_bounds__(Cfg::THREADS, Cfg::MIN_BLOCKS)
           const int64_t part =
               ((static_cast<int64_t>(U.split) * p.batch + U.b) * p.n_heads + U.h) * p.t_q + row_glob;
           if (p.kv_splits > 1) {
-            float4* dst = reinterpret_cast<float4*>(p.ws_o + part * DH);
+            float4* dst = p.merge ? reinterpret_cast<float4*>(merge_o + srow * DH)
+                                  : reinterpret_cast<float4*>(p.ws_o + part * DH);
 #pragma unroll
             for (int v = 0; v < DH / 4; ++v) dst[v] = make_float4(0.f, 0.f, 0.f, 0.f);
-            reinterpret_cast<float2*>(p.ws_ml)[part] = make_float2(-INFINITY, 0.f);
+            (p.merge ? merge_ml[srow] : reinterpret_cast<float2*>(p.ws_ml)[part]) = make_float2(-INFINITY, 0.f);
           } else {
             uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<int64_t>(U.b) * p.t_q + row_glob) * p.out_stride +
                                                   U.h * DH);
@@ -637,7 +647,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, Cfg::MIN_BLOCKS)
         }
         if (!row_ok) continue;
         if (p.kv_splits > 1) {
-          float4* dst = reinterpret_cast<float4*>(p.ws_o + part * DH + c * 32);
+          float4* dst = p.merge ? reinterpret_cast<float4*>(merge_o + srow * DH + c * 32)
+                                : reinterpret_cast<float4*>(p.ws_o + part * DH + c * 32);
 #pragma unroll
           for (int v = 0; v < 8; ++v)
             dst[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
@@ -656,13 +667,60 @@ __global__ void __launch_bounds__(Cfg::THREADS, Cfg::MIN_BLOCKS)
           }
         }
       }
-      if (row_ok && p.kv_splits > 1) reinterpret_cast<float2*>(p.ws_ml)[part] = make_float2(m_run, l_run);
+      if (row_ok && p.kv_splits > 1)
+        (p.merge ? merge_ml[srow] : reinterpret_cast<float2*>(p.ws_ml)[part]) = make_float2(m_run, l_run);
     }
   }
 
   __syncwarp();
   tc_fence_before();
   __syncthreads();
+  if (p.merge) {
+    // Every CTA of the cluster holds one split's partial of the same query
+    // tile. CTA r writes rows r, r + C, r + 2C, ... of the output from all C
+    // partials (read through the cluster's shared-memory window):
+    //   M = max_s m_s,  L = sum_s l_s 2^(m_s - M) [+ 2^(sink*log2e - M)],
+    //   o = sum_s O_s 2^(m_s - M) / L.
+    cluster_sync();
+    if (warp < C::SOFTMAX_WARPS) {
+      const Unit U = decode_unit<EXT>(p, blockIdx.x);
+      const int nc = p.kv_splits;  // cluster size
+      const int r = static_cast<int>(cluster_ctarank());
+      const uint32_t o_base = smem_u32(merge_o), ml_base = smem_u32(merge_ml);
+      for (int i = r + nc * warp; i < U.rows; i += nc * C::SOFTMAX_WARPS) {
+        float m_s = -INFINITY, l_s = 0.f;
+        if (lane < nc) {
+          const float2 ml = ld_shared_cluster_f2(mapa_shared(ml_base + i * 8, lane));
+          m_s = ml.x;
+          l_s = ml.y;
+        }
+        float mx = l_s > 0.f ? m_s : -INFINITY;
+#pragma unroll
+        for (int off = 4; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        mx = __shfl_sync(0xffffffffu, mx, 0);
+        const float w = (l_s > 0.f && mx != -INFINITY) ? ex2_approx(m_s - mx) : 0.f;
+        float lw = l_s * w;
+#pragma unroll
+        for (int off = 4; off > 0; off >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, off);
+        float l = __shfl_sync(0xffffffffu, lw, 0);
+        float o0 = 0.f, o1 = 0.f;
+        for (int sp = 0; sp < nc; ++sp) {
+          const float ws = __shfl_sync(0xffffffffu, w, sp);
+          const float2 ov = ld_shared_cluster_f2(mapa_shared(o_base + (i * DH + 2 * lane) * 4, sp));
+          o0 += ov.x * ws;
+          o1 += ov.y * ws;
+        }
+        if constexpr (EXT) {
+          if (p.sinks != nullptr && mx != -INFINITY) l += ex2_approx(__ldg(p.sinks + U.h) * kLog2e - mx);
+        }
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        __half2* dst = reinterpret_cast<__half2*>(p.out + (static_cast<int64_t>(U.b) * p.t_q + U.q0 + i) * p.out_stride +
+                                                  U.h * DH);
+        dst[lane] = __floats2half2_rn(o0 * inv, o1 * inv);
+      }
+    }
+    cluster_sync();  // no CTA leaves while another still reads its partial
+  }
   if (warp == C::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);

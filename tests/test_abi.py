@@ -90,7 +90,7 @@ def test_forward_rejects_bad_masks(lib):
     assert call_forward(lib, mask=mk, t_kv=64) == attn.ATTN_ERR_INVALID         # 1 word < 64 slots
     mk = attn.AttnMask(); mk.kind = attn.MASK_SLOTMASK; mk.bits = P4 + 0x1000002; mk.words_per_row = 2
     assert call_forward(lib, mask=mk, t_kv=64) == attn.ATTN_ERR_INVALID         # misaligned bits
-    mk = attn.AttnMask(); mk.kind = attn.MASK_FULL; mk.reserved = 1
+    mk = attn.AttnMask(); mk.kind = attn.MASK_FULL; mk.flags = 2
     assert call_forward(lib, mask=mk) == attn.ATTN_ERR_INVALID
 
 
@@ -231,7 +231,21 @@ def test_plan_splits_short_query_blocks(lib, kind, t_q, t_kv, heads, sms):
     assert p["kv_splits"] * p["kv_tiles_per_split"] >= n_kv > (p["kv_splits"] - 1) * p["kv_tiles_per_split"]
     assert p["units"] == base * splits
     rows = splits * heads * t_q
-    assert p["workspace_bytes"] == rows * 64 * 4 + rows * 2 * 4  # partial O, then (m, l)
+    if splits <= 8:  # merged inside a cluster of `splits` CTAs: no workspace
+        assert p["cluster_merge"] == 1 and p["workspace_bytes"] == 0
+    else:
+        assert p["cluster_merge"] == 0
+        assert p["workspace_bytes"] == rows * 64 * 4 + rows * 2 * 4  # partial O, then (m, l)
+
+
+def test_plan_long_splits_use_the_workspace(lib):
+    # one head of 80 queries over 12000 keys: 94 key tiles over up to 148 CTAs
+    p = attn.debug_plan(1, 80, 12000, 1, attn.MASK_FULL, num_sms=148)
+    assert p["kv_splits"] > 8 and p["cluster_merge"] == 0
+    assert p["workspace_bytes"] == p["kv_splits"] * 80 * (64 * 4 + 2 * 4)
+    # the verify block's cross-attention: 6 splits, merged in clusters
+    p = attn.debug_plan(1, 80, 1500, 20, attn.MASK_FULL, num_sms=148)
+    assert (p["kv_splits"], p["cluster_merge"], p["workspace_bytes"]) == (6, 1, 0)
 
 
 def test_plan_does_not_split_when_units_fill_the_gpu(lib):

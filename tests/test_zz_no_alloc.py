@@ -3,14 +3,17 @@ device memory (a host that owns every device allocation through its own pool,
 or a real-time decode loop that must not allocate between frames).
 
 It runs the split-KV cross-attention with its partials in the library's fixed
-device array instead of a caller workspace. Two calls with different queries,
-enqueued back to back on one stream with no synchronisation between them
-(the second reuses the array the first one wrote), must each match the FP64
-oracle and the workspace entry point attn_cross within the parity tolerance;
+device array instead of a caller workspace (splits of more than 8 parts; up to
+8 parts merge inside a thread-block cluster and need no scratch). Two calls
+with different queries on such a shape, enqueued back to back on one stream
+with no synchronisation between them (the second reuses the array the first
+one wrote), must each match the FP64 oracle and the workspace entry point
+attn_cross within the parity tolerance;
 a call after a warm-up must allocate no device memory; and a shape whose
 split needs more than the fixed 4 MiB must be refused. This file is named to
 be collected last."""
 import ctypes
+import types
 
 import numpy as np
 import pytest
@@ -28,11 +31,22 @@ def _mat(t):
     return attn.AttnMat(ctypes.c_void_p(t.data_ptr()), t.stride(0))
 
 
+class _Shape:
+    """The verify block's 80 queries over 12000 encoder frames with 2 heads:
+    long enough a key range that the split takes more than 8 parts, so it
+    keeps its partials in scratch memory (shorter splits merge inside a
+    thread-block cluster and need none)."""
+    t_q, t_enc, n_heads, d_model = 80, 12000, 2, 128
+
+
 def _verify_cross_inputs():
-    spec = inputs.VERIFY_WORKLOADS["verify"]
-    inp = inputs.make_verify_inputs(spec)
+    spec = _Shape()
+    rng = np.random.default_rng(5)
+    inp = types.SimpleNamespace(q=inputs.random_f16(rng, (spec.t_q, spec.d_model)),
+                                k_enc=inputs.random_f16(rng, (spec.t_enc, spec.d_model)),
+                                v_enc=inputs.random_f16(rng, (spec.t_enc, spec.d_model)))
     # a second block of queries, so the two calls' partials differ
-    q2 = inputs.random_f16(np.random.default_rng([spec.seed, 99]), inp.q.shape)
+    q2 = inputs.random_f16(np.random.default_rng([5, 99]), inp.q.shape)
     return spec, inp, q2
 
 
@@ -44,9 +58,12 @@ def test_static_scratch_matches_oracle_and_workspace_entry_point_back_to_back():
     ke, ve = to_dev(inp.k_enc), to_dev(inp.v_enc)
     qs = [to_dev(inp.q), to_dev(q2_host)]
     d = spec.d_model
-    # the shape splits its key range, so the scratch is really used
+    # the shape splits its key range into more parts than a cluster merges,
+    # so the scratch is really used
     need = attn.workspace_size(1, spec.t_q, spec.t_enc, spec.n_heads, attn.MASK_FULL)
     assert 0 < need <= STATIC_SCRATCH_BYTES
+    assert attn.debug_plan(1, spec.t_q, spec.t_enc, spec.n_heads, attn.MASK_FULL,
+                           num_sms=torch.cuda.get_device_properties(0).multi_processor_count)["kv_splits"] > 8
 
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     outs = [torch.full((spec.t_q, d), float("nan"), dtype=torch.float16, device="cuda") for _ in qs]
@@ -89,8 +106,9 @@ def test_static_scratch_allocates_nothing():
 def test_static_scratch_refuses_splits_larger_than_the_array():
     import torch
     lib = attn.load_library()
-    # 70 query tiles of one head: the split plan needs 2 x 8960 x 264 bytes > 4 MiB
-    t_q, t_enc, heads = 128 * 70, 300, 1
+    # 16 query tiles of one head over 18 key tiles: 9 splits (more than a
+    # cluster merges), whose partials need 9 x 2048 x 264 bytes > 4 MiB
+    t_q, t_enc, heads = 128 * 16, 2304, 1
     rng = np.random.default_rng(0)
     q = to_dev(inputs.random_f16(rng, (t_q, 64)))
     k = to_dev(inputs.random_f16(rng, (t_enc, 64)))
