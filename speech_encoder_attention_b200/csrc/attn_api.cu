@@ -69,6 +69,28 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
   return g_encode;
 }
 
+// Raises the dynamic shared-memory limit of the attention kernel's four
+// variants with a K/V ring of ST stages.
+template <int ST>
+bool set_attention_smem() {
+  constexpr int bytes = sea::fa::CfgT<ST>::SMEM_BYTES;
+  return cudaFuncSetAttribute(sea::fa::flash_attn_kernel<false, false, ST>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess &&
+         cudaFuncSetAttribute(sea::fa::flash_attn_kernel<false, true, ST>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess &&
+         cudaFuncSetAttribute(sea::fa::flash_attn_kernel<true, false, ST>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess &&
+         cudaFuncSetAttribute(sea::fa::flash_attn_kernel<true, true, ST>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+}
+
+// The attention kernel variant for a mask family, the options and the ring depth.
+template <int ST>
+auto attention_kernel(bool slot, bool ext) {
+  return slot ? (ext ? sea::fa::flash_attn_kernel<true, true, ST> : sea::fa::flash_attn_kernel<true, false, ST>)
+              : (ext ? sea::fa::flash_attn_kernel<false, true, ST> : sea::fa::flash_attn_kernel<false, false, ST>);
+}
+
 // Per-device set-up: checks for an sm_100 part, records the SM count and the
 // error-word address, and raises the dynamic shared-memory limits once.
 attn_status device_info(DeviceInfo** out) {
@@ -97,14 +119,7 @@ attn_status device_info(DeviceInfo** out) {
                              sea::gemm::PairShape::SMEM_BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(sea::q8::qkv_q8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              sea::q8::SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(sea::fa::flash_attn_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             sea::fa::Cfg::SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(sea::fa::flash_attn_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             sea::fa::Cfg::SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(sea::fa::flash_attn_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             sea::fa::Cfg::SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(sea::fa::flash_attn_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             sea::fa::Cfg::SMEM_BYTES) != cudaSuccess ||
+        !set_attention_smem<2>() || !set_attention_smem<4>() ||
         cudaFuncSetAttribute(sea::fr::flash_range_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              sea::fr::Cfg::SMEM_BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(sea::fr::flash_range_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -417,16 +432,21 @@ attn_status launch_attention(attn_mat q, attn_mat k, attn_mat v, int32_t batch, 
   const bool ext = p.mask_kind == sea::fa::kBand || p.causal != 0 || p.q_lens != nullptr ||
                    p.kv_lens != nullptr || p.sinks != nullptr;
   const int threads = sea::fa::Cfg::THREADS;
-  const int smem = sea::fa::Cfg::SMEM_BYTES;
   cudaError_t err;
   // A merged split runs one unit per CTA, the splits of a query tile (units
   // next to each other) forming one cluster.
   const unsigned cluster = pl.merge ? static_cast<unsigned>(pl.kv_splits) : 1u;
-  if (slot || pl.merge) {
+  // At most one CTA per SM: a four-stage K/V ring (a short unit's key tiles
+  // all load at once); otherwise two CTAs per SM with two stages each.
+  const bool deep = units <= dev->num_sms;
+  if (slot || pl.merge || (deep && !kRangeKernelV2)) {
     // One unit per CTA (SLOTMASK: its tile flags need a pass over every row's words).
-    auto kern = slot ? (ext ? sea::fa::flash_attn_kernel<true, true> : sea::fa::flash_attn_kernel<true, false>)
-                     : (ext ? sea::fa::flash_attn_kernel<false, true> : sea::fa::flash_attn_kernel<false, false>);
-    err = launch_pdl_cluster(kern, dim3(p.units), dim3(threads), smem, stream, cluster, tq, tk, tv, p);
+    if (deep)
+      err = launch_pdl_cluster(attention_kernel<4>(slot, ext), dim3(p.units), dim3(threads),
+                               sea::fa::CfgT<4>::SMEM_BYTES, stream, cluster, tq, tk, tv, p);
+    else
+      err = launch_pdl_cluster(attention_kernel<2>(slot, ext), dim3(p.units), dim3(threads),
+                               sea::fa::CfgT<2>::SMEM_BYTES, stream, cluster, tq, tk, tv, p);
   } else if (kRangeKernelV2) {
     // Persistent: one CTA per SM walks the units.
     using FR = sea::fr::Cfg;
@@ -440,10 +460,8 @@ attn_status launch_attention(attn_mat q, attn_mat k, attn_mat v, int32_t batch, 
   } else {
     // Persistent: Cfg::MIN_BLOCKS CTAs per SM walk the units.
     const int grid = static_cast<int>(std::min<int64_t>(units, int64_t(sea::fa::Cfg::MIN_BLOCKS) * dev->num_sms));
-    if (ext)
-      err = launch_pdl(sea::fa::flash_attn_kernel<false, true>, dim3(grid), dim3(threads), smem, stream, tq, tk, tv, p);
-    else
-      err = launch_pdl(sea::fa::flash_attn_kernel<false, false>, dim3(grid), dim3(threads), smem, stream, tq, tk, tv, p);
+    err = launch_pdl(attention_kernel<2>(false, ext), dim3(grid), dim3(threads), sea::fa::Cfg::SMEM_BYTES, stream, tq,
+                     tk, tv, p);
   }
   if (err != cudaSuccess) return ATTN_ERR_CUDA;
   if (pl.kv_splits > 1 && !pl.merge) {

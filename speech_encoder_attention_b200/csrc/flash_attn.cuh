@@ -86,14 +86,18 @@ struct Params {
   uint64_t limit_ns;
 };
 
-struct Cfg {
+// STAGES_: K/V ring depth. Two stages (99.5 KB of shared memory) let two CTAs
+// share an SM; launches of at most one CTA per SM (short query blocks) take
+// four, so a unit's first four key tiles load at once.
+template <int STAGES_ = 2>
+struct CfgT {
   static constexpr int SOFTMAX_WARPS = 4;
   static constexpr int SOFTMAX_THREADS = 128;
   static constexpr int PRODUCER_WARP = 4;
   static constexpr int MMA_WARP = 5;
   static constexpr int THREADS = 192;
-  static constexpr int MIN_BLOCKS = 2;  // two CTAs per SM
-  static constexpr int STAGES = 2;      // K/V ring depth
+  static constexpr int MIN_BLOCKS = 2;  // two CTAs per SM (with two stages)
+  static constexpr int STAGES = STAGES_;
   static constexpr int TMEM_COLS = 256;
   static constexpr uint32_t S_COL = 0;    // 128 fp32 columns
   static constexpr uint32_t O_COL = 128;  // 64 fp32 columns
@@ -109,6 +113,7 @@ struct Cfg {
   static constexpr int OFF_MISC = OFF_FLAGS + 4 * MAX_FLAG_WORDS;
   static constexpr int SMEM_BYTES = 1024 + OFF_MISC + 16;
 };
+using Cfg = CfgT<2>;
 
 // Lazy rescaling: the exponent reference m only moves when a row's max grows
 // by more than this (log2 units), so p <= 2^15 fits fp16 and O is rescaled rarely.
@@ -244,11 +249,11 @@ __device__ __forceinline__ Unit decode_unit(const Params& p, int u) {
 // (FULL, CHUNK, BAND, with lengths and causal) carries no bitmask code and runs persistent CTAs. SLOTMASK
 // CTAs each own one unit (gridDim.x == units): the tile flags need one pass of
 // every row's mask words before any role starts.
-template <bool SLOT, bool EXT>
-__global__ void __launch_bounds__(Cfg::THREADS, Cfg::MIN_BLOCKS)
+template <bool SLOT, bool EXT, int STAGES = 2>
+__global__ void __launch_bounds__(CfgT<STAGES>::THREADS, STAGES == 2 ? 2 : 1)
     flash_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const Params p) {
-  using C = Cfg;
+  using C = CfgT<STAGES>;
   constexpr int ST = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -291,6 +296,11 @@ __global__ void __launch_bounds__(Cfg::THREADS, Cfg::MIN_BLOCKS)
     mbar_init(drain_bar, 1);
     *abort_flag = 0u;
     fence_barrier_init();
+    // The tensor maps are launch parameters, not the previous kernel's data:
+    // fetch them before waiting for that kernel.
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
   }
   if (threadIdx.x < MAX_FLAG_WORDS) flags[threadIdx.x] = 0u;
   if (warp == C::MMA_WARP) {
@@ -313,8 +323,16 @@ __global__ void __launch_bounds__(Cfg::THREADS, Cfg::MIN_BLOCKS)
   float2* merge_ml = reinterpret_cast<float2*>(smem + C::OFF_K + BQ * DH * 4);
 
   // SLOTMASK: mark the key tiles any row of this CTA's (single) unit may see.
+  // The producer starts the unit's Q load first: Q does not depend on the
+  // flags, and the pass waits on the mask words' global-memory latency.
+  bool q_preloaded = false;
   if constexpr (use_flags) {
     const Unit U = decode_unit<EXT>(p, blockIdx.x);
+    if (warp == C::PRODUCER_WARP && lane == 0 && U.rows > 0) {
+      mbar_arrive_expect_tx(q_full(0), TILE_BYTES);
+      tma_load_3d(sbase + C::OFF_Q, &tm_q, q_full(0), U.h * DH, U.q0, U.b);
+      q_preloaded = true;
+    }
     if (warp < C::SOFTMAX_WARPS && srow < U.rows) {
       const uint32_t* mrow = p.bits + static_cast<int64_t>(U.q0 + srow) * p.words_per_row;
       for (int j = U.j_begin; j < U.j_end; ++j) {
@@ -333,18 +351,17 @@ __global__ void __launch_bounds__(Cfg::THREADS, Cfg::MIN_BLOCKS)
   if (warp == C::PRODUCER_WARP) {
     if (lane == 0) {
       // ---------------- TMA producer ----------------
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
       int qn = 0, it = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
         const Unit U = decode_unit<EXT>(p, u);
         if (U.rows == 0 || (!SLOT && U.j_end <= U.j_begin)) continue;  // see the softmax's empty-unit note
         const int qb = qn & 1;
-        if (!mbar_wait(q_empty(qb), ((qn >> 1) & 1) ^ 1u, wc)) break;
-        mbar_arrive_expect_tx(q_full(qb), TILE_BYTES);
-        tma_load_3d(sbase + C::OFF_Q + qb * TILE_BYTES, &tm_q, q_full(qb), U.h * DH, U.q0, U.b);
+        if (!(q_preloaded && qn == 0)) {
+          if (!mbar_wait(q_empty(qb), ((qn >> 1) & 1) ^ 1u, wc)) break;
+          mbar_arrive_expect_tx(q_full(qb), TILE_BYTES);
+          tma_load_3d(sbase + C::OFF_Q + qb * TILE_BYTES, &tm_q, q_full(qb), U.h * DH, U.q0, U.b);
+        }
         ++qn;
         for (int j = U.j_begin; j < U.j_end; ++j) {
           if (!tile_on(j)) continue;
@@ -681,42 +698,58 @@ __global__ void __launch_bounds__(Cfg::THREADS, Cfg::MIN_BLOCKS)
     // partials (read through the cluster's shared-memory window):
     //   M = max_s m_s,  L = sum_s l_s 2^(m_s - M) [+ 2^(sink*log2e - M)],
     //   o = sum_s O_s 2^(m_s - M) / L.
+    // A thread takes one 4-column chunk of one row at a time and issues the
+    // loads of all C partials before using any, so each item costs one round
+    // trip through the cluster.
     cluster_sync();
-    if (warp < C::SOFTMAX_WARPS) {
+    {
       const Unit U = decode_unit<EXT>(p, blockIdx.x);
-      const int nc = p.kv_splits;  // cluster size
+      const int nc = p.kv_splits;  // cluster size, at most 8
       const int r = static_cast<int>(cluster_ctarank());
+      const int own = U.rows > r ? (U.rows - r + nc - 1) / nc : 0;  // rows this CTA writes
       const uint32_t o_base = smem_u32(merge_o), ml_base = smem_u32(merge_ml);
-      for (int i = r + nc * warp; i < U.rows; i += nc * C::SOFTMAX_WARPS) {
-        float m_s = -INFINITY, l_s = 0.f;
-        if (lane < nc) {
-          const float2 ml = ld_shared_cluster_f2(mapa_shared(ml_base + i * 8, lane));
-          m_s = ml.x;
-          l_s = ml.y;
-        }
-        float mx = l_s > 0.f ? m_s : -INFINITY;
+      float sink_l2 = -INFINITY;
+      if constexpr (EXT) {
+        if (p.sinks != nullptr) sink_l2 = __ldg(p.sinks + U.h) * kLog2e;
+      }
+      for (int item = threadIdx.x; item < own * (DH / 4); item += C::THREADS) {
+        const int i = r + nc * (item / (DH / 4));  // tile row
+        const int c4 = item % (DH / 4);             // 4-column chunk
+        float2 ml[8];
+        float4 ov[8];
 #pragma unroll
-        for (int off = 4; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        mx = __shfl_sync(0xffffffffu, mx, 0);
-        const float w = (l_s > 0.f && mx != -INFINITY) ? ex2_approx(m_s - mx) : 0.f;
-        float lw = l_s * w;
-#pragma unroll
-        for (int off = 4; off > 0; off >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, off);
-        float l = __shfl_sync(0xffffffffu, lw, 0);
-        float o0 = 0.f, o1 = 0.f;
-        for (int sp = 0; sp < nc; ++sp) {
-          const float ws = __shfl_sync(0xffffffffu, w, sp);
-          const float2 ov = ld_shared_cluster_f2(mapa_shared(o_base + (i * DH + 2 * lane) * 4, sp));
-          o0 += ov.x * ws;
-          o1 += ov.y * ws;
+        for (int sp = 0; sp < 8; ++sp) {
+          if (sp < nc) {
+            ml[sp] = ld_shared_cluster_f2(mapa_shared(ml_base + i * 8, sp));
+            ov[sp] = ld_shared_cluster_f4(mapa_shared(o_base + (i * DH + 4 * c4) * 4, sp));
+          }
         }
-        if constexpr (EXT) {
-          if (p.sinks != nullptr && mx != -INFINITY) l += ex2_approx(__ldg(p.sinks + U.h) * kLog2e - mx);
+        float mx = -INFINITY;
+#pragma unroll
+        for (int sp = 0; sp < 8; ++sp)
+          if (sp < nc && ml[sp].y > 0.f) mx = fmaxf(mx, ml[sp].x);
+        float l = 0.f;
+        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (mx != -INFINITY) {
+#pragma unroll
+          for (int sp = 0; sp < 8; ++sp) {
+            if (sp < nc && ml[sp].y > 0.f) {
+              const float w = ex2_approx(ml[sp].x - mx);
+              l += ml[sp].y * w;
+              o.x += ov[sp].x * w;
+              o.y += ov[sp].y * w;
+              o.z += ov[sp].z * w;
+              o.w += ov[sp].w * w;
+            }
+          }
+          if (sink_l2 != -INFINITY) l += ex2_approx(sink_l2 - mx);
         }
         const float inv = l > 0.f ? 1.f / l : 0.f;
-        __half2* dst = reinterpret_cast<__half2*>(p.out + (static_cast<int64_t>(U.b) * p.t_q + U.q0 + i) * p.out_stride +
-                                                  U.h * DH);
-        dst[lane] = __floats2half2_rn(o0 * inv, o1 * inv);
+        uint2 h;
+        h.x = pack_half2(o.x * inv, o.y * inv);
+        h.y = pack_half2(o.z * inv, o.w * inv);
+        *reinterpret_cast<uint2*>(p.out + (static_cast<int64_t>(U.b) * p.t_q + U.q0 + i) * p.out_stride + U.h * DH +
+                                  4 * c4) = h;
       }
     }
     cluster_sync();  // no CTA leaves while another still reads its partial

@@ -214,6 +214,11 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     mbar_init(drain_bar, 1);
     *abort_flag = 0u;
     fence_barrier_init();
+    // The tensor maps are launch parameters, not the previous kernel's data:
+    // fetch them before waiting for that kernel.
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
   }
   if (warp == C::MMA_WARP) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
@@ -235,9 +240,6 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   if (warp == C::PRODUCER_WARP) {
     if (lane == 0) {
       // ---------------- TMA producer ----------------
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
       int nu = 0, it = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
