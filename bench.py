@@ -22,6 +22,7 @@ copied back inside the timed region.
 from __future__ import annotations
 
 import argparse
+import contextlib
 import hashlib
 import json
 import re
@@ -235,6 +236,7 @@ def relaunch_under_torchrun(n: int, argv):
 
 class EncoderStep:
     """Packed projection + attention over a batch of windows (or chunks)."""
+    cold = False  # L2 flushed before each step; every launch between events
 
     def __init__(self, spec: inputs.EncoderSpec, device):
         import torch
@@ -260,6 +262,9 @@ class EncoderStep:
         self.launches_per_step = 2
 
     def run(self, events=None):
+        # Direct launches: a CUDA graph of the two calls measured ~9 us slower
+        # per step than these (programmatic launch of the attention grid
+        # during the projection's last wave).
         a, d, s = self.attn, self.d, self.spec
         if events:
             events[0].record()
@@ -296,39 +301,91 @@ class EncoderStep:
         return {"frames": self.spec.batch * self.spec.t}
 
 
-class GraphedCalls:
-    """A step's library calls, each captured once in its own CUDA graph and
-    replayed every step. The decode-side calls take microseconds on the GPU,
-    less than the host spends per call (argument marshalling, three tensor-map
-    encodings, the launch); launched directly, that host time would show up as
-    device idle time between the timing events. Replaying a graph per call
-    leaves one event between consecutive calls, so each call is still timed
-    on its own."""
+class StepGraphs:
+    """A decode-side step's library calls captured in CUDA graphs, over N
+    device copies of the step's buffers.
 
-    def __init__(self, calls):
+    Each copy's step is one graph: its calls back to back, as a decode loop or
+    an encoder pipeline captures them (one launch per call, programmatic
+    launches between them). A second set of graphs, one per copy and call,
+    times the calls one at a time (an event between consecutive calls).
+
+    A decode-side step reads 6-12 MB, far less than the 126 MB L2, so a flush
+    write between its steps would also evict the kernels' code and constants,
+    which a decode loop finds in L2. Instead such a step's inputs and outputs
+    exist N times with N x (bytes of one copy) >= 2 x L2: step i uses copy
+    i mod N, whose data was last touched N - 1 steps (more than twice the L2's
+    capacity of other data) earlier, so it comes from HBM again."""
+
+    def __init__(self, make_calls, n_copies):
         import torch
-        for fn in calls:  # warm-up: per-device set-up and lazy module loading
-            fn()
-        torch.cuda.synchronize()
-        self.graphs = []
-        for fn in calls:
+        self.n = n_copies
+        self.step_graphs, self.call_graphs = [], []
+        for i in range(n_copies):
+            calls = make_calls(i)
+            for fn in calls:  # warm-up: per-device set-up and lazy module loading
+                fn()
+            torch.cuda.synchronize()
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
-                fn()
-            self.graphs.append(g)
+                for fn in calls:
+                    fn()
+            self.step_graphs.append(g)
+            per_call = []
+            for fn in calls:
+                gc = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gc):
+                    fn()
+                per_call.append(gc)
+            self.call_graphs.append(per_call)
         torch.cuda.synchronize()
+        self.i = 0
 
-    def run(self, events=None):
-        for i, g in enumerate(self.graphs):
-            if events:
-                events[i].record()
-            g.replay()
+    def next_copy(self) -> int:
+        i = self.i % self.n
+        self.i += 1
+        return i
+
+    def run(self, events=None, copy=None):
+        """One step on the next copy (or the given one); events = [start, end]."""
+        g = self.step_graphs[self.next_copy() if copy is None else copy]
         if events:
-            events[len(self.graphs)].record()
+            events[0].record()
+        g.replay()
+        if events:
+            events[-1].record()
+
+    def run_split(self, events):
+        """One step on the next copy, an event before each call and after the last."""
+        graphs = self.call_graphs[self.next_copy()]
+        for k, g in enumerate(graphs):
+            events[k].record()
+            g.replay()
+        events[len(graphs)].record()
+
+
+def cold_copy_count(device, bytes_per_copy: int) -> int:
+    import torch
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    return max(2, -(-2 * l2 // max(1, bytes_per_copy)))
+
+
+STEP_TIMING_COLD = ("each step one CUDA graph; ms_per_step = K steps back to back between two events / K; "
+                    "latency_ms_one_step = a second pass with events around each step; per-kernel times = "
+                    "a third pass of per-call graphs with an event between calls")
+STEP_TIMING_FLUSHED = ("direct launches with an event before, between and after them; L2 flushed before each "
+                       "step outside the events")
+COLD_L2_NOTE = ("not flushed: inputs and outputs rotate over device copies totalling more than 2 x L2, "
+                "so each step reads its data from HBM; one CUDA graph per step")
+
+
+def cold_note(n_copies: int, bytes_per_copy: int) -> dict:
+    return {"copies": n_copies, "bytes_per_copy": bytes_per_copy, "total_bytes": n_copies * bytes_per_copy}
 
 
 class VerifyStep:
     """Token-tree self-attention (SLOTMASK) plus cross-attention of the same block."""
+    cold = True
 
     def __init__(self, spec: inputs.VerifySpec, device):
         import torch
@@ -336,16 +393,21 @@ class VerifyStep:
         self.attn = attn
         self.spec = spec
         inp = inputs.make_verify_inputs(spec)
-        dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
-        self.q, self.kc, self.vc = dev(inp.q), dev(inp.k_cache), dev(inp.v_cache)
-        self.ke, self.ve = dev(inp.k_enc), dev(inp.v_enc)
-        self.bits = dev(inp.bits.view(np.int32))
         d = spec.d_model
-        self.o_self = torch.empty(spec.t_q, d, dtype=torch.float16, device=device)
-        self.o_cross = torch.empty(spec.t_q, d, dtype=torch.float16, device=device)
         ws = max(attn.workspace_size(1, spec.t_q, spec.slots, spec.n_heads, attn.MASK_SLOTMASK),
                  attn.workspace_size(1, spec.t_q, spec.t_enc, spec.n_heads, attn.MASK_FULL))
-        self.ws = torch.empty(max(ws, 16), dtype=torch.uint8, device=device)
+        host = {"q": inp.q, "kc": inp.k_cache, "vc": inp.v_cache, "ke": inp.k_enc, "ve": inp.v_enc,
+                "bits": inp.bits.view(np.int32)}
+        per_copy = sum(a.nbytes for a in host.values()) + 2 * (2 * spec.t_q * d) + ws
+        n = cold_copy_count(device, per_copy)
+        self.copies = []
+        for _ in range(n):
+            c = {k: torch.from_numpy(np.ascontiguousarray(v)).to(device) for k, v in host.items()}
+            c["o_self"] = torch.empty(spec.t_q, d, dtype=torch.float16, device=device)
+            c["o_cross"] = torch.empty(spec.t_q, d, dtype=torch.float16, device=device)
+            c["ws"] = torch.empty(max(ws, 16), dtype=torch.uint8, device=device)
+            self.copies.append(c)
+        self.cold_copies = cold_note(n, per_copy)
         self.host_q = torch.from_numpy(inp.q).pin_memory()
         self.host_out = torch.empty(2 * spec.t_q, d, dtype=torch.float16).pin_memory()
         pairs = int(inputs.unpack_bits(inp.bits, spec.slots).sum())
@@ -364,22 +426,31 @@ class VerifyStep:
                  attn.debug_plan(1, spec.t_q, spec.t_enc, spec.n_heads, attn.MASK_FULL, num_sms=sms))
         self.launches_per_step = sum(1 + (pl["kv_splits"] > 1 and not pl["cluster_merge"]) for pl in plans)
         a, s = self.attn, self.spec
-        self.graphed = GraphedCalls([
-            lambda: a.attn_forward(self.q, self.kc, self.vc, 1, s.t_q, s.slots, s.n_heads,
-                                   mask_kind=a.MASK_SLOTMASK, bits=self.bits, out=self.o_self, workspace=self.ws),
-            lambda: a.attn_cross(self.q, self.ke, self.ve, 1, s.t_q, s.t_enc, s.n_heads, out=self.o_cross,
-                                 workspace=self.ws)])
+
+        def calls(i):
+            c = self.copies[i]
+            return [lambda: a.attn_forward(c["q"], c["kc"], c["vc"], 1, s.t_q, s.slots, s.n_heads,
+                                           mask_kind=a.MASK_SLOTMASK, bits=c["bits"], out=c["o_self"],
+                                           workspace=c["ws"]),
+                    lambda: a.attn_cross(c["q"], c["ke"], c["ve"], 1, s.t_q, s.t_enc, s.n_heads, out=c["o_cross"],
+                                         workspace=c["ws"])]
+        self.graphs = StepGraphs(calls, n)
 
     def run(self, events=None):
-        self.graphed.run(events)
+        self.graphs.run(events)
+
+    def run_split(self, events):
+        self.graphs.run_split(events)
 
     def run_e2e(self, events=None):
+        i = self.graphs.next_copy()
+        c = self.copies[i]
         if events:
             events[0].record()
-        self.q.copy_(self.host_q, non_blocking=True)
-        self.run()
-        self.host_out[:self.spec.t_q].copy_(self.o_self, non_blocking=True)
-        self.host_out[self.spec.t_q:].copy_(self.o_cross, non_blocking=True)
+        c["q"].copy_(self.host_q, non_blocking=True)
+        self.graphs.run(copy=i)
+        self.host_out[:self.spec.t_q].copy_(c["o_self"], non_blocking=True)
+        self.host_out[self.spec.t_q:].copy_(c["o_cross"], non_blocking=True)
         if events:
             events[-1].record()
 
@@ -404,6 +475,7 @@ class VerifyStep:
 class DrafterStep:
     """The drafter's block attention: each beam's 16 queries at the end of its
     448 keys, bidirectional or causal inside the block, with per-head sinks."""
+    cold = True
 
     def __init__(self, spec: inputs.DrafterSpec, device):
         import torch
@@ -411,12 +483,18 @@ class DrafterStep:
         self.attn = attn
         self.spec = spec
         inp = inputs.make_drafter_inputs(spec)
-        dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
-        self.q, self.k, self.v, self.sinks = dev(inp.q), dev(inp.k), dev(inp.v), dev(inp.sinks)
         d = spec.d_model
-        self.out = torch.empty(spec.beams * spec.t_q, d, dtype=torch.float16, device=device)
         ws = attn.workspace_size(spec.beams, spec.t_q, spec.t_kv, spec.n_heads, attn.MASK_FULL)
-        self.ws = torch.empty(max(ws, 16), dtype=torch.uint8, device=device)
+        host = {"q": inp.q, "k": inp.k, "v": inp.v, "sinks": inp.sinks}
+        per_copy = sum(a.nbytes for a in host.values()) + 2 * spec.beams * spec.t_q * d + ws
+        n = cold_copy_count(device, per_copy)
+        self.copies = []
+        for _ in range(n):
+            c = {k: torch.from_numpy(np.ascontiguousarray(v)).to(device) for k, v in host.items()}
+            c["out"] = torch.empty(spec.beams * spec.t_q, d, dtype=torch.float16, device=device)
+            c["ws"] = torch.empty(max(ws, 16), dtype=torch.uint8, device=device)
+            self.copies.append(c)
+        self.cold_copies = cold_note(n, per_copy)
         self.split_launches = 2 if ws > 0 else 1
         self.host_q = torch.from_numpy(inp.q).pin_memory()
         self.host_out = torch.empty(spec.beams * spec.t_q, d, dtype=torch.float16).pin_memory()
@@ -426,21 +504,28 @@ class DrafterStep:
         self.flops = {"drafter_attn": attn_pair_flops(spec.beams * per_beam, spec.n_heads)}
         self.bytes = {"drafter_attn": 2 * d * spec.beams * (2 * spec.t_q + 2 * spec.t_kv) + 4 * spec.n_heads}
         self.launches_per_step = self.split_launches
-
         a, s = self.attn, self.spec
-        self.graphed = GraphedCalls([
-            lambda: a.attn_forward(self.q, self.k, self.v, s.beams, s.t_q, s.t_kv, s.n_heads, causal=s.causal,
-                                   sinks=self.sinks, out=self.out, workspace=self.ws)])
+
+        def calls(i):
+            c = self.copies[i]
+            return [lambda: a.attn_forward(c["q"], c["k"], c["v"], s.beams, s.t_q, s.t_kv, s.n_heads,
+                                           causal=s.causal, sinks=c["sinks"], out=c["out"], workspace=c["ws"])]
+        self.graphs = StepGraphs(calls, n)
 
     def run(self, events=None):
-        self.graphed.run(events)
+        self.graphs.run(events)
+
+    def run_split(self, events):
+        self.graphs.run_split(events)
 
     def run_e2e(self, events=None):
+        i = self.graphs.next_copy()
+        c = self.copies[i]
         if events:
             events[0].record()
-        self.q.copy_(self.host_q, non_blocking=True)
-        self.run()
-        self.host_out.copy_(self.out, non_blocking=True)
+        c["q"].copy_(self.host_q, non_blocking=True)
+        self.graphs.run(copy=i)
+        self.host_out.copy_(c["out"], non_blocking=True)
         if events:
             events[-1].record()
 
@@ -464,6 +549,7 @@ class DrafterStep:
 
 class Q8Step:
     """The decoder's packed projection with Q8_0 weights (one launch)."""
+    cold = True
 
     def __init__(self, spec: inputs.Q8Spec, device):
         import torch
@@ -471,10 +557,16 @@ class Q8Step:
         self.attn = attn
         self.spec = spec
         inp = inputs.make_q8_inputs(spec)
-        dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
-        self.x, self.w, self.bq, self.bv = dev(inp.x), dev(inp.w_blocks), dev(inp.b_q), dev(inp.b_v)
         d = spec.d_model
-        self.out = torch.empty(spec.rows, 3 * d, dtype=torch.float16, device=device)
+        host = {"x": inp.x, "w": inp.w_blocks, "bq": inp.b_q, "bv": inp.b_v}
+        per_copy = sum(a.nbytes for a in host.values()) + 2 * spec.rows * 3 * d
+        n = cold_copy_count(device, per_copy)
+        self.copies = []
+        for _ in range(n):
+            c = {k: torch.from_numpy(np.ascontiguousarray(v)).to(device) for k, v in host.items()}
+            c["out"] = torch.empty(spec.rows, 3 * d, dtype=torch.float16, device=device)
+            self.copies.append(c)
+        self.cold_copies = cold_note(n, per_copy)
         self.host_x = torch.from_numpy(inp.x).pin_memory()
         self.host_out = torch.empty(spec.rows, 3 * d, dtype=torch.float16).pin_memory()
         self.kernels = ["q8_proj"]
@@ -482,18 +574,25 @@ class Q8Step:
         self.bytes = {"q8_proj": inp.w_blocks.nbytes + 2 * spec.rows * d + 2 * spec.rows * 3 * d}
         self.launches_per_step = 1
 
-        self.graphed = GraphedCalls([
-            lambda: self.attn.attn_qkv_pack_q8_0(self.x, self.w, self.bq, self.bv, out=self.out)])
+        def calls(i):
+            c = self.copies[i]
+            return [lambda: self.attn.attn_qkv_pack_q8_0(c["x"], c["w"], c["bq"], c["bv"], out=c["out"])]
+        self.graphs = StepGraphs(calls, n)
 
     def run(self, events=None):
-        self.graphed.run(events)
+        self.graphs.run(events)
+
+    def run_split(self, events):
+        self.graphs.run_split(events)
 
     def run_e2e(self, events=None):
+        i = self.graphs.next_copy()
+        c = self.copies[i]
         if events:
             events[0].record()
-        self.x.copy_(self.host_x, non_blocking=True)
-        self.run()
-        self.host_out.copy_(self.out, non_blocking=True)
+        c["x"].copy_(self.host_x, non_blocking=True)
+        self.graphs.run(copy=i)
+        self.host_out.copy_(c["out"], non_blocking=True)
         if events:
             events[-1].record()
 
@@ -691,18 +790,18 @@ def workload_config(spec):
         return {"workload": f"{spec.name}: packed projection of {spec.rows} decoder rows, d_model {spec.d_model}, "
                             f"Q8_0 weights [{3 * spec.d_model} x {spec.d_model}]",
                 "rows": spec.rows, "d_model": spec.d_model, "weights": "Q8_0 (34-byte blocks)",
-                "l2": "flushed between timed steps (256 MiB write)", "parallelism": "replicas (weak)"}
+                "l2": COLD_L2_NOTE, "parallelism": "replicas (weak)"}
     if isinstance(spec, inputs.DrafterSpec):
         return {"workload": f"{spec.name}: {spec.beams} beams x {spec.t_q} queries at the end of {spec.t_kv} keys, "
                             f"{'causal' if spec.causal else 'bidirectional'} block, per-head sinks, "
                             f"{spec.n_heads}x64 heads",
                 "beams": spec.beams, "t_q": spec.t_q, "t_kv": spec.t_kv, "causal": spec.causal,
-                "n_heads": spec.n_heads, "l2": "flushed between timed steps (256 MiB write)",
+                "n_heads": spec.n_heads, "l2": COLD_L2_NOTE,
                 "parallelism": "replicas (weak)"}
     return {"workload": f"{spec.name}: {spec.t_q} query rows ({spec.beams} beams x {spec.block}) over a "
                         f"{spec.slots}-slot token-tree cache + cross-attention to {spec.t_enc} encoder frames",
             "t_q": spec.t_q, "slots": spec.slots, "t_enc": spec.t_enc, "n_heads": spec.n_heads,
-            "l2": "flushed between timed steps (256 MiB write)", "parallelism": "replicas (weak)"}
+            "l2": COLD_L2_NOTE, "parallelism": "replicas (weak)"}
 
 
 # ---------------------------------------------------------------------------
@@ -717,26 +816,77 @@ def check_device_errors(step, where):
         raise RuntimeError(f"device error word {word:#x} after the {where}: a kernel wait timed out")
 
 
+def time_steps(step, flush, steps, warmup, clocks=None, barrier=None):
+    """Warm-up, then `steps` timed steps.
+
+    step.cold (a decode-side step: one CUDA graph per step, buffers rotating
+    over copies larger than L2, no flush): the K steps run back to back
+    between two events, as the base contract times them; a second pass
+    brackets each step with its own events (the latency of one step, graph
+    launch included); a third replays per-call graphs with an event between
+    calls (the per-kernel times).
+    Otherwise (the encoder): L2 is flushed (a 256 MiB write) before each step,
+    outside its events, and an event sits before, between and after the
+    step's launches.
+    Returns (mean step ms, [mean ms per kernel], mean one-step latency ms or None)."""
+    import torch
+    cold = getattr(step, "cold", False)
+    nk = len(step.kernels)
+    new_events = lambda n: [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    for _ in range(warmup):
+        if not cold:
+            flush.zero_()
+        step.run()
+        if cold:
+            step.run_split(new_events(nk + 1))
+    torch.cuda.synchronize()
+    block = new_events(2)
+    ev = [new_events(2 if cold else nk + 1) for _ in range(steps)]
+    if barrier is not None:
+        barrier()
+    torch.cuda.synchronize()
+    with (clocks if clocks is not None else contextlib.nullcontext()):
+        if cold:
+            block[0].record()
+            for _ in range(steps):
+                step.run()
+            block[1].record()
+        else:
+            for e in ev:
+                flush.zero_()
+                step.run(e)
+        torch.cuda.synchronize()
+    if barrier is not None:
+        barrier()
+    if not cold:
+        step_ms = sum(e[0].elapsed_time(e[-1]) for e in ev) / steps
+        per_kernel = [sum(e[k].elapsed_time(e[k + 1]) for e in ev) / steps for k in range(nk)]
+        return step_ms, per_kernel, None
+    step_ms = block[0].elapsed_time(block[1]) / steps
+    for e in ev:
+        step.run(e)
+    torch.cuda.synchronize()
+    latency_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
+    ev = [new_events(nk + 1) for _ in range(steps)]
+    for e in ev:
+        step.run_split(e)
+    torch.cuda.synchronize()
+    per_kernel = [sum(e[k].elapsed_time(e[k + 1]) for e in ev) / steps for k in range(nk)]
+    return step_ms, per_kernel, latency_ms
+
+
 def time_secondary(name, device, steps, warmup, ws):
     """The bandwidth-bound verify step (token-tree SLOTMASK + cross-attention),
-    timed like the main step (L2 flushed between steps, CUDA events on the
+    timed like a `--workload verify` run (data cold in HBM, CUDA events on the
     launching stream, max over ranks): its step time, algorithmic bytes and
     fraction of the HBM roofline."""
     import torch
     step = make_step(name, device)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
-    for _ in range(warmup):
-        step.run()
-    torch.cuda.synchronize()
-    nk = len(step.kernels)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(steps)]
-    for e in ev:
-        flush.zero_()
-        step.run(e)
-    torch.cuda.synchronize()
+    local_ms, per_kernel, latency_ms = time_steps(step, flush, steps, warmup)
     check_device_errors(step, f"{name} steps")
-    local_ms = sum(e[0].elapsed_time(e[nk]) for e in ev) / steps
     ms = reduce_step_time(local_ms, device)
+    latency_ms = reduce_step_time(latency_ms, device)
     peaks, peak_kind = load_peaks()
     total_bytes = step.total_bytes()
     gbs = total_bytes / (ms * 1e-3) / 1e9
@@ -744,9 +894,10 @@ def time_secondary(name, device, steps, warmup, ws):
             "algorithmic_bytes_per_step": total_bytes, "achieved_gbs": gbs, "peak_gbs": peaks["hbm_gbs"],
             "hbm_frac": gbs / peaks["hbm_gbs"], "peak_source": f"{peak_kind} hbm_gbs",
             "tflops": step.total_flops() / (ms * 1e-3) / 1e12,
-            "kernels_us": {k: sum(e[i].elapsed_time(e[i + 1]) for e in ev) / steps * 1e3
-                           for i, k in enumerate(step.kernels)},
-            "launches_per_step": step.launches_per_step}
+            "kernels_us": {k: per_kernel[i] * 1e3 for i, k in enumerate(step.kernels)},
+            "latency_ms_one_step": latency_ms,
+            "launches_per_step": step.launches_per_step, "cold_copies": step.cold_copies,
+            "timing": STEP_TIMING_COLD}
 
 
 def run_gpu(args):
@@ -761,38 +912,19 @@ def run_gpu(args):
                                 device_id=device)
     step = make_step(args.workload, device)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
-    stream = torch.cuda.current_stream()
-    nk = len(step.kernels)
-
-    for _ in range(args.warmup):
-        step.run()
-    torch.cuda.synchronize()
-
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(args.steps)]
 
     def barrier():
         if ws > 1:
             import torch.distributed as dist
             dist.barrier()
 
-    barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clocks:
-        for i in range(args.steps):
-            flush.zero_()
-            step.run(ev[i])
-        torch.cuda.synchronize()
-    barrier()
+    clocks = ClockSampler(local)
+    local_ms, per_kernel, latency_ms = time_steps(step, flush, args.steps, args.warmup, clocks, barrier)
     check_device_errors(step, "timed steps")
-    per_kernel = np.zeros(nk)
-    step_ms = 0.0
-    for e in ev:
-        for k in range(nk):
-            per_kernel[k] += e[k].elapsed_time(e[k + 1])
-        step_ms += e[0].elapsed_time(e[nk])
-    local_ms = step_ms / args.steps
-    per_kernel /= args.steps
+    per_kernel = np.asarray(per_kernel)
     ms = reduce_step_time(local_ms, device)
+    if latency_ms is not None:
+        latency_ms = reduce_step_time(latency_ms, device)
 
     # end to end through the same calls, host buffers, copies inside the timed region
     e2e_ms = None
@@ -830,12 +962,21 @@ def run_gpu(args):
     value = whole_job_rate(flops, ws, ms) / 1e12
     top = int(np.argmax(per_kernel))
     kname = step.kernels[top]
+    clock_rec = clocks.summary()
+    # The burst peak for a kernel timed in a short run, the sustained one
+    # (a seconds-long loop under the power cap) once the power cap acted
+    # during the timed steps.
+    capped = "sw_power_cap" in (clock_rec or {}).get("reasons", [])
+    tensor_key = "bf16_tflops_sustained" if capped and "bf16_tflops_sustained" in peaks else "bf16_tflops"
     if is_encoder:
-        peak = peaks["bf16_tflops"]
+        peak = peaks[tensor_key]
         achieved = step.flops[kname] / (per_kernel[top] * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": stored_traffic(kname, args.workload),
-                "kernel": kname, "peak_source": f"{peak_kind} bf16_tflops (burst); fp16 dense rate = bf16 rate",
+                "frac": achieved / peak, "frac_of_burst_peak": achieved / peaks["bf16_tflops"],
+                "traffic": stored_traffic(kname, args.workload), "kernel": kname,
+                "peak_source": (f"{peak_kind} {tensor_key} "
+                                + ("(sustained: sw_power_cap active during the timed steps)" if capped
+                                   else "(burst)") + "; fp16 dense rate = bf16 rate"),
                 "algorithmic_flops_per_launch": step.flops[kname], "launch_us": per_kernel[top] * 1e3}
         unit = "TFLOP/s"
     else:
@@ -864,6 +1005,8 @@ def run_gpu(args):
         "vs_baseline": None, "dtype": "f16", "data": "synthetic (seeded; random-init weights)",
         "config": workload_config(spec),
         "pct_of_peak": 100.0 * value / (peaks["bf16_tflops"] * ws),
+        **({"pct_of_sustained_peak": 100.0 * value / (peaks["bf16_tflops_sustained"] * ws)}
+           if is_encoder and "bf16_tflops_sustained" in peaks else {}),
         "units_per_s": {k: v * ws / (ms * 1e-3) for k, v in step.units().items()},
         "roofline": roof,
         "kernels": all_kernels,
@@ -874,7 +1017,10 @@ def run_gpu(args):
             "ms_per_step": e2e_ms},
         "secondary": secondary,
         "gpu_launches": step.launches_per_step * args.steps,
-        "clocks": clocks.summary(),
+        "timing": STEP_TIMING_COLD if getattr(step, "cold", False) else STEP_TIMING_FLUSHED,
+        **({"cold_copies": step.cold_copies, "latency_ms_one_step": latency_ms}
+           if getattr(step, "cold", False) else {}),
+        "clocks": clock_rec,
         "kernel_source_hash": kernel_source_hash(),
     }
     print(json.dumps(line), flush=True)
