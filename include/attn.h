@@ -267,6 +267,10 @@ attn_status attn_debug_error_word(attn_stream_t stream, uint32_t *word_out);
  *   kv_splits, kv_tiles_per_split: the key split (1 = none); units = work units
  *   workspace_bytes: what attn_workspace_size would report for that device
  *   cluster_merge: 1 when the split parts merge inside a cluster (no workspace)
+ *   narrow: 1 when query tiles of at most 32 rows are computed in the narrow
+ *     layout (the rows in each of the four tensor-memory lane quadrants, each
+ *     softmax warp a quarter of every key tile's columns, the four partials
+ *     merged per row): range masks, no split, at most one unit per SM
  *   proj_tile_n: the projection's output tile for proj_rows rows of d_model:
  *     256 or 192 (128-row tiles of that width on one SM), 512 (256 x 256
  *     tiles on a pair of SMs), 0 when proj_rows or d_model is 0
@@ -281,6 +285,7 @@ typedef struct {
   int64_t units;
   size_t workspace_bytes;
   int32_t cluster_merge;
+  int32_t narrow;
 } attn_plan_info;
 
 attn_status attn_debug_plan(int32_t batch, int32_t t_q, int32_t t_kv, int32_t n_heads, int32_t mask_kind,

@@ -69,6 +69,7 @@ class AttnPlanInfo(ctypes.Structure):
         ("units", ctypes.c_int64),
         ("workspace_bytes", ctypes.c_size_t),
         ("cluster_merge", ctypes.c_int32),
+        ("narrow", ctypes.c_int32),
     ]
 
 

@@ -13,7 +13,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libattn.so")
 SOURCES = ["attn_api.cu"]
-HEADERS = ["attn_api.cu", "flash_attn.cuh", "flash_range.cuh", "qkv_gemm.cuh", "qkv_q8.cuh", "sm100_ptx.cuh"]
+HEADERS = ["attn_api.cu", "flash_attn.cuh", "qkv_gemm.cuh", "qkv_q8.cuh", "sm100_ptx.cuh"]
 
 
 def nvcc() -> str:

@@ -16,7 +16,6 @@
 
 #include "attn.h"
 #include "flash_attn.cuh"
-#include "flash_range.cuh"
 #include "qkv_gemm.cuh"
 #include "qkv_q8.cuh"
 #include "sm100_ptx.cuh"
@@ -81,7 +80,11 @@ bool set_attention_smem() {
          cudaFuncSetAttribute(sea::fa::flash_attn_kernel<true, false, ST>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess &&
          cudaFuncSetAttribute(sea::fa::flash_attn_kernel<true, true, ST>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess &&
+         (ST != 4 || (cudaFuncSetAttribute(sea::fa::flash_attn_kernel<false, false, 4, true>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess &&
+                      cudaFuncSetAttribute(sea::fa::flash_attn_kernel<false, true, 4, true>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess));
 }
 
 // The attention kernel variant for a mask family, the options and the ring depth.
@@ -89,6 +92,11 @@ template <int ST>
 auto attention_kernel(bool slot, bool ext) {
   return slot ? (ext ? sea::fa::flash_attn_kernel<true, true, ST> : sea::fa::flash_attn_kernel<true, false, ST>)
               : (ext ? sea::fa::flash_attn_kernel<false, true, ST> : sea::fa::flash_attn_kernel<false, false, ST>);
+}
+
+// The narrow-tile variant (range family, four stages).
+auto narrow_attention_kernel(bool ext) {
+  return ext ? sea::fa::flash_attn_kernel<false, true, 4, true> : sea::fa::flash_attn_kernel<false, false, 4, true>;
 }
 
 // Per-device set-up: checks for an sm_100 part, records the SM count and the
@@ -119,11 +127,7 @@ attn_status device_info(DeviceInfo** out) {
                              sea::gemm::PairShape::SMEM_BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(sea::q8::qkv_q8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              sea::q8::SMEM_BYTES) != cudaSuccess ||
-        !set_attention_smem<2>() || !set_attention_smem<4>() ||
-        cudaFuncSetAttribute(sea::fr::flash_range_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             sea::fr::Cfg::SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(sea::fr::flash_range_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             sea::fr::Cfg::SMEM_BYTES) != cudaSuccess)
+        !set_attention_smem<2>() || !set_attention_smem<4>())
       return ATTN_ERR_CUDA;
     d.num_sms = sms;
     d.err = static_cast<uint32_t*>(err);
@@ -177,12 +181,12 @@ bool encode_q8_rows(CUtensorMap* m, const void* ptr, uint64_t units_per_row, uin
 // (columns, frames, sequence) view of a [batch*t, >=cols] matrix: rows past a
 // sequence's end read as zeros instead of the next sequence's frames.
 bool encode_seq_3d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t t, uint64_t batch,
-                   uint64_t row_stride_elems) {
+                   uint64_t row_stride_elems, uint32_t box_rows = 128) {
   auto enc = encoder();
   if (!enc) return false;
   cuuint64_t dims[3] = {cols, t, batch};
   cuuint64_t strides[2] = {row_stride_elems * 2, row_stride_elems * 2 * t};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -242,6 +246,14 @@ FaPlan plan_forward(int batch, int t_q, int t_kv, int n_heads, int mask_kind, in
   return pl;
 }
 
+// Query tiles of at most 32 rows with no key split and at most one unit per
+// SM take the narrow layout (the rows in every lane quadrant, each softmax
+// warp a quarter of the key columns); the range masks only.
+bool narrow_tiles(const FaPlan& pl, int mask_kind, int64_t units, int num_sms) {
+  return mask_kind != sea::fa::kSlotmask && pl.kv_splits == 1 && pl.tiles_per_seg == 1 && pl.seg_len <= 32 &&
+         units <= num_sms;
+}
+
 // Launches with programmatic stream serialization: the kernel may start its
 // prologue while the previous kernel in the stream finishes; every kernel of
 // this library waits (griddepcontrol.wait) before it touches global memory.
@@ -276,12 +288,6 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return launch_pdl_cluster(kernel, grid, block, smem, stream, 1u, std::forward<Args>(args)...);
 }
 
-// The range masks (FULL, CHUNK, BAND and their options) run on the one-CTA-
-// per-SM kernel of flash_range.cuh when set, else on flash_attn.cuh's.
-#ifndef SEA_RANGE_KERNEL_V2
-#define SEA_RANGE_KERNEL_V2 0
-#endif
-constexpr bool kRangeKernelV2 = SEA_RANGE_KERNEL_V2 != 0;
 
 // Row counts from which the projection runs on CTA pairs (256 x 256 tiles,
 // cta_group::2): large enough that the pair tiles fill the GPU.
@@ -369,11 +375,6 @@ attn_status launch_attention(attn_mat q, attn_mat k, attn_mat v, int32_t batch, 
     pl.merge = false;
     pl.ws_bytes = 0;
   }
-  if (pl.merge && mask.kind != ATTN_MASK_SLOTMASK && kRangeKernelV2) {
-    pl.merge = false;  // that kernel writes its partials to the workspace only
-    const size_t rows = static_cast<size_t>(pl.kv_splits) * batch * n_heads * t_q;
-    pl.ws_bytes = rows * sea::fa::DH * sizeof(float) + rows * 2 * sizeof(float);
-  }
   if (pl.kv_splits > 1 && !pl.merge) {
     if (workspace == nullptr) {
       pl.kv_splits = 1;  // caller opted out of the split: same result, one CTA per key range
@@ -384,8 +385,12 @@ attn_status launch_attention(attn_mat q, attn_mat k, attn_mat v, int32_t batch, 
     }
   }
 
+  const int64_t units = static_cast<int64_t>(batch) * n_heads * pl.q_tiles * pl.kv_splits;
+  if (units > INT32_MAX) return ATTN_ERR_INVALID;
+  const bool narrow = narrow_tiles(pl, mask.kind == ATTN_MASK_SLOTMASK ? sea::fa::kSlotmask : sea::fa::kFull, units,
+                                   dev->num_sms);
   CUtensorMap tq, tk, tv;
-  if (!encode_seq_3d(&tq, q.ptr, cols, t_q, batch, q.row_stride) ||
+  if (!encode_seq_3d(&tq, q.ptr, cols, t_q, batch, q.row_stride, narrow ? 32 : 128) ||
       !encode_seq_3d(&tk, k.ptr, cols, t_kv, batch, k.row_stride) ||
       !encode_seq_3d(&tv, v.ptr, cols, t_kv, batch, v.row_stride))
     return ATTN_ERR_CUDA;
@@ -424,8 +429,6 @@ attn_status launch_attention(attn_mat q, attn_mat k, attn_mat v, int32_t batch, 
   p.err = dev->err;
   p.limit_ns = sea::kDefaultTimeoutNs;
 
-  const int64_t units = static_cast<int64_t>(batch) * n_heads * pl.q_tiles * pl.kv_splits;
-  if (units > INT32_MAX) return ATTN_ERR_INVALID;
   p.units = static_cast<int>(units);
   const bool slot = p.mask_kind == sea::fa::kSlotmask;
   // The lengths / causal / BAND / sinks code is compiled into its own variant.
@@ -439,7 +442,10 @@ attn_status launch_attention(attn_mat q, attn_mat k, attn_mat v, int32_t batch, 
   // At most one CTA per SM: a four-stage K/V ring (a short unit's key tiles
   // all load at once); otherwise two CTAs per SM with two stages each.
   const bool deep = units <= dev->num_sms;
-  if (slot || pl.merge || (deep && !kRangeKernelV2)) {
+  if (narrow) {
+    err = launch_pdl(narrow_attention_kernel(ext), dim3(p.units), dim3(threads), sea::fa::CfgT<4>::SMEM_BYTES, stream,
+                     tq, tk, tv, p);
+  } else if (slot || deep) {
     // One unit per CTA (SLOTMASK: its tile flags need a pass over every row's words).
     if (deep)
       err = launch_pdl_cluster(attention_kernel<4>(slot, ext), dim3(p.units), dim3(threads),
@@ -447,16 +453,6 @@ attn_status launch_attention(attn_mat q, attn_mat k, attn_mat v, int32_t batch, 
     else
       err = launch_pdl_cluster(attention_kernel<2>(slot, ext), dim3(p.units), dim3(threads),
                                sea::fa::CfgT<2>::SMEM_BYTES, stream, cluster, tq, tk, tv, p);
-  } else if (kRangeKernelV2) {
-    // Persistent: one CTA per SM walks the units.
-    using FR = sea::fr::Cfg;
-    const int grid = static_cast<int>(std::min<int64_t>(units, dev->num_sms));
-    if (ext)
-      err = launch_pdl(sea::fr::flash_range_kernel<true>, dim3(grid), dim3(FR::THREADS), FR::SMEM_BYTES, stream, tq, tk,
-                       tv, p);
-    else
-      err = launch_pdl(sea::fr::flash_range_kernel<false>, dim3(grid), dim3(FR::THREADS), FR::SMEM_BYTES, stream, tq,
-                       tk, tv, p);
   } else {
     // Persistent: Cfg::MIN_BLOCKS CTAs per SM walk the units.
     const int grid = static_cast<int>(std::min<int64_t>(units, int64_t(sea::fa::Cfg::MIN_BLOCKS) * dev->num_sms));
@@ -694,6 +690,9 @@ attn_status attn_debug_plan(int32_t batch, int32_t t_q, int32_t t_kv, int32_t n_
   out->units = static_cast<int64_t>(batch) * n_heads * pl.q_tiles * pl.kv_splits;
   out->workspace_bytes = pl.ws_bytes;
   out->cluster_merge = pl.merge ? 1 : 0;
+  out->narrow = narrow_tiles(pl, kind == ATTN_MASK_SLOTMASK ? sea::fa::kSlotmask : sea::fa::kFull, out->units, num_sms)
+                    ? 1
+                    : 0;
   out->proj_tile_n = (proj_rows > 0 && d_model > 0) ? gemm_tile_n(proj_rows, 3 * static_cast<int64_t>(d_model), num_sms)
                                                     : 0;
   return ATTN_OK;

@@ -107,8 +107,9 @@ struct CfgT {
   static constexpr int OFF_V = OFF_K + STAGES * TILE_BYTES;
   static constexpr int OFF_BARS = OFF_V + STAGES * TILE_BYTES;
   // q_full[2], q_empty[2], k_full[S], v_full[S], kv_empty[S], s_full, s_free,
-  // p_full, o_done, o_free, drain
-  static constexpr int NUM_BARS = 4 + 3 * STAGES + 6;
+  // p_full, o_done, o_free, drain, quarters (narrow tiles: the four warps'
+  // partials are in shared memory)
+  static constexpr int NUM_BARS = 4 + 3 * STAGES + 7;
   static constexpr int OFF_FLAGS = OFF_BARS + 8 * NUM_BARS;
   static constexpr int OFF_MISC = OFF_FLAGS + 4 * MAX_FLAG_WORDS;
   static constexpr int SMEM_BYTES = 1024 + OFF_MISC + 16;
@@ -120,13 +121,6 @@ using Cfg = CfgT<2>;
 constexpr float RESCALE_LIMIT = 15.0f;
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Bit k set: pair k of every 16 keys takes the FMA-pipe exp2 instead
-// of MUFU ex2. Measured on B200 the extra instructions cost more than the
-// MUFU relief buys in this kernel, so no pair is moved.
-#ifndef SEA_POLY_PAIRS
-#define SEA_POLY_PAIRS 0x00u
-#endif
-constexpr uint32_t POLY_PAIRS = SEA_POLY_PAIRS;
 
 struct TileGeom {
   int q0;     // first query row (sequence-local)
@@ -249,12 +243,24 @@ __device__ __forceinline__ Unit decode_unit(const Params& p, int u) {
 // (FULL, CHUNK, BAND, with lengths and causal) carries no bitmask code and runs persistent CTAs. SLOTMASK
 // CTAs each own one unit (gridDim.x == units): the tile flags need one pass of
 // every row's mask words before any role starts.
-template <bool SLOT, bool EXT, int STAGES = 2>
+//
+// NARROW (query tiles of at most 32 rows, one unit per CTA, no key split):
+// the tile's rows are loaded four times, into rows 0, 32, 64 and 96 of the Q
+// buffer, so every softmax warp holds all of them in its own tensor-memory
+// lane quadrant, and warp w takes key columns [32w, 32w + 32) of each key
+// tile. Each warp keeps its own running max, sum and O over its quarter of
+// the keys (its P columns outside the quarter stay zero, so P V sums only
+// its keys); the epilogue merges the four partials through shared memory as
+// a split-KV merge does. A thread then exponentiates 32 scores per key tile
+// instead of 128, which shortens the per-tile chain of a decode-sized block.
+template <bool SLOT, bool EXT, int STAGES = 2, bool NARROW = false>
 __global__ void __launch_bounds__(CfgT<STAGES>::THREADS, STAGES == 2 ? 2 : 1)
     flash_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const Params p) {
   using C = CfgT<STAGES>;
   constexpr int ST = C::STAGES;
+  static_assert(!(SLOT && NARROW), "narrow tiles serve the range masks only");
+  constexpr int NC = NARROW ? 32 : BKV;  // score columns a softmax thread holds per key tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -270,6 +276,7 @@ __global__ void __launch_bounds__(CfgT<STAGES>::THREADS, STAGES == 2 ? 2 : 1)
   const uint32_t o_done = s_full + 24u;
   const uint32_t o_free = s_full + 32u;
   const uint32_t drain_bar = s_full + 40u;
+  const uint32_t quarters_bar = s_full + 48u;
   uint32_t* flags = reinterpret_cast<uint32_t*>(smem + C::OFF_FLAGS);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + C::OFF_MISC + 4);
@@ -294,6 +301,7 @@ __global__ void __launch_bounds__(CfgT<STAGES>::THREADS, STAGES == 2 ? 2 : 1)
     mbar_init(o_done, 1);
     mbar_init(o_free, 4);
     mbar_init(drain_bar, 1);
+    mbar_init(quarters_bar, 4);
     *abort_flag = 0u;
     fence_barrier_init();
     // The tensor maps are launch parameters, not the previous kernel's data:
@@ -332,6 +340,12 @@ __global__ void __launch_bounds__(CfgT<STAGES>::THREADS, STAGES == 2 ? 2 : 1)
       mbar_arrive_expect_tx(q_full(0), TILE_BYTES);
       tma_load_3d(sbase + C::OFF_Q, &tm_q, q_full(0), U.h * DH, U.q0, U.b);
       q_preloaded = true;
+      // Which key tiles load is known only after the pass; meanwhile pull the
+      // first ones into L2.
+      for (int j = U.j_begin; j < min(U.j_end, U.j_begin + ST); ++j) {
+        tma_prefetch_l2_3d(&tm_k, U.h * DH, U.kv_lo + j * BKV, U.b);
+        tma_prefetch_l2_3d(&tm_v, U.h * DH, U.kv_lo + j * BKV, U.b);
+      }
     }
     if (warp < C::SOFTMAX_WARPS && srow < U.rows) {
       const uint32_t* mrow = p.bits + static_cast<int64_t>(U.q0 + srow) * p.words_per_row;
@@ -360,7 +374,15 @@ __global__ void __launch_bounds__(CfgT<STAGES>::THREADS, STAGES == 2 ? 2 : 1)
         if (!(q_preloaded && qn == 0)) {
           if (!mbar_wait(q_empty(qb), ((qn >> 1) & 1) ^ 1u, wc)) break;
           mbar_arrive_expect_tx(q_full(qb), TILE_BYTES);
-          tma_load_3d(sbase + C::OFF_Q + qb * TILE_BYTES, &tm_q, q_full(qb), U.h * DH, U.q0, U.b);
+          if constexpr (NARROW) {
+            // tm_q's box is 32 rows here: the same rows into each lane quadrant
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+              tma_load_3d(sbase + C::OFF_Q + qb * TILE_BYTES + r * (TILE_BYTES / 4), &tm_q, q_full(qb), U.h * DH,
+                          U.q0, U.b);
+          } else {
+            tma_load_3d(sbase + C::OFF_Q + qb * TILE_BYTES, &tm_q, q_full(qb), U.h * DH, U.q0, U.b);
+          }
         }
         ++qn;
         for (int j = U.j_begin; j < U.j_end; ++j) {
@@ -472,13 +494,25 @@ __global__ void __launch_bounds__(CfgT<STAGES>::THREADS, STAGES == 2 ? 2 : 1)
     const uint32_t o_tmem = tmem_base + C::O_COL + lane_field;
     const uint32_t p_tmem = tmem_base + C::P_COL + lane_field;
     const float sl2 = p.scale_log2;
+    // NARROW: this warp's key columns of each tile start at cb; its P columns
+    // outside them stay zero for the CTA's life.
+    const int cb = NARROW ? 32 * (warp & 3) : 0;
+    if constexpr (NARROW) {
+      uint32_t z[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) z[e] = 0u;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) tmem_st8_async(p_tmem + c * 8, z);
+      tmem_wait_st();
+    }
     int it = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
       const Unit U = decode_unit<EXT>(p, u);
       if (U.rows == 0) continue;
-      const int row_glob = U.q0 + srow;  // sequence-local query row
-      const bool row_ok = srow < U.rows;
+      const int qrow = NARROW ? lane : srow;  // row within the query tile
+      const int row_glob = U.q0 + qrow;       // sequence-local query row
+      const bool row_ok = qrow < U.rows;
       if (!SLOT && U.j_end <= U.j_begin) {
         // No key tile (padding rows, rows before the first key, a split past
         // the unit's keys): the rows see no key. In the persistent kernel such
@@ -486,7 +520,7 @@ __global__ void __launch_bounds__(CfgT<STAGES>::THREADS, STAGES == 2 ? 2 : 1)
         // the softmax cannot complete barrier phases ahead of the MMA thread's
         // parity waits. (A SLOTMASK CTA owns one unit: its empty unit takes
         // the general path.)
-        if (row_ok) {
+        if (row_ok && (!NARROW || (warp & 3) == 0)) {
           const int64_t part =
               ((static_cast<int64_t>(U.split) * p.batch + U.b) * p.n_heads + U.h) * p.t_q + row_glob;
           if (p.kv_splits > 1) {
@@ -519,19 +553,22 @@ __global__ void __launch_bounds__(CfgT<STAGES>::THREADS, STAGES == 2 ? 2 : 1)
           break;
         }
         tc_fence_after();
-        float s[128];
+        float s[NC];
         {
-          uint32_t r[128];
-          tmem_ld128(s_tmem, r);
+          uint32_t r[NC];
+          if constexpr (NARROW)
+            tmem_ld32(s_tmem + cb, r);
+          else
+            tmem_ld128(s_tmem, r);
 #pragma unroll
-          for (int e = 0; e < 128; ++e) s[e] = __uint_as_float(r[e]);
+          for (int e = 0; e < NC; ++e) s[e] = __uint_as_float(r[e]);
         }
         // S is in registers: the next tile's S may overwrite it.
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(s_free);
 
-        const int kv0 = U.kv_lo + j * BKV;  // key index of s[0]
+        const int kv0 = U.kv_lo + j * BKV + cb;  // key index of s[0]
         if constexpr (use_flags) {
           uint32_t wbits[4];
 #pragma unroll
@@ -546,48 +583,42 @@ __global__ void __launch_bounds__(CfgT<STAGES>::THREADS, STAGES == 2 ? 2 : 1)
         } else {
           const int a = lo_i - kv0;
           const int bnd = hi_i - kv0;
-          if (a > 0 || bnd < BKV) {
+          if (a > 0 || bnd < NC) {
 #pragma unroll
-            for (int e = 0; e < 128; ++e)
+            for (int e = 0; e < NC; ++e)
               if (e < a || e >= bnd) s[e] = -INFINITY;
           }
         }
-        // The tile's row max: eight independent chains of 3-input max.
+        // The tile's row max: four independent chains of 3-input max.
         auto row_max = [&]() -> float {
           float mx4[4];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) mx4[i] = fmaxf(s[i], s[124 + i]);
+          for (int i = 0; i < 4; ++i) mx4[i] = fmaxf(s[i], s[NC - 4 + i]);
 #pragma unroll
-          for (int e = 4; e < 124; e += 8) {
+          for (int e = 4; e < NC - 4; e += 8) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) mx4[i] = fmax3(mx4[i], s[e + i], s[e + 4 + i]);
           }
           return fmaxf(fmax3(mx4[0], mx4[1], mx4[2]), mx4[3]);
         };
-        // p = 2^(s*scale*log2e - m), summed in fp32 and written to P as fp16
-        // pairs, 32 keys at a time. MUFU ex2 serves 16 lanes per clock per SM;
-        // pairs picked by POLY_PAIRS take the FMA-pipe exp2 instead.
+        // p = 2^(s*scale*log2e - m) on MUFU ex2 (16 lanes per clock per SM),
+        // summed in fp32 and written to P as fp16 pairs, 16 keys at a time.
         auto exp_tile = [&](float m_use) -> float {
           const uint64_t sl2x2 = f2_pack(sl2, sl2);
           const uint64_t negm2 = f2_pack(-m_use, -m_use);
           uint64_t acc2[2] = {0ull, 0ull};
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
+          for (int c = 0; c < NC / 16; ++c) {
             uint32_t pk[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-              float x0, x1, p0, p1;
+              float x0, x1;
               f2_unpack(f2_fma(f2_pack(s[16 * c + 2 * i], s[16 * c + 2 * i + 1]), sl2x2, negm2), x0, x1);
-              if ((POLY_PAIRS >> i) & 1) {
-                exp2_poly_x2(x0, x1, p0, p1);
-              } else {
-                p0 = ex2_approx(x0);
-                p1 = ex2_approx(x1);
-              }
+              const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
               acc2[i & 1] = f2_add(acc2[i & 1], f2_pack(p0, p1));
               pk[i] = pack_half2(p0, p1);
             }
-            tmem_st8_async(p_tmem + c * 8, pk);
+            tmem_st8_async(p_tmem + cb / 2 + c * 8, pk);
           }
           tmem_wait_st();
           float sum0, sum1;
@@ -639,6 +670,95 @@ __global__ void __launch_bounds__(CfgT<STAGES>::THREADS, STAGES == 2 ? 2 : 1)
       const bool have_o = t_unit > 0 && mbar_wait(o_done, (it - 1) & 1, wc);
       if (t_unit > 0 && !have_o) ok = false;
       if (have_o) tc_fence_after();
+      if constexpr (NARROW) {
+        // The four warps' partials of the tile's rows, merged through shared
+        // memory (the K/V stages: this CTA's only unit has no load or MMA
+        // left once its last P V is done):
+        //   M = max_w m_w,  L = sum_w l_w 2^(m_w - M) [+ 2^(sink*log2e - M)],
+        //   o = sum_w O_w 2^(m_w - M) / L.
+        // Slot row w*32 + r holds warp w's partial of row r; its 16-byte
+        // chunks are rotated by (r mod 16) against bank conflicts.
+        float* q_o = reinterpret_cast<float*>(smem + C::OFF_K);
+        float2* q_ml = reinterpret_cast<float2*>(smem + C::OFF_K + 4 * 32 * DH * 4);
+        const int slot_row = (warp & 3) * 32 + lane;
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+          uint32_t r[32];
+          if (have_o) {
+            tmem_ld32(o_tmem + c * 32, r);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = 0u;
+          }
+          if (c == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(o_free);
+          }
+          float4* dst = reinterpret_cast<float4*>(q_o + slot_row * DH);
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            dst[(c * 8 + v) ^ (lane & 15)] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                                         __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+        }
+        q_ml[slot_row] = make_float2(m_run, have_o ? l_run : 0.f);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(quarters_bar);
+        if (!mbar_wait(quarters_bar, 0, wc)) {
+          ok = false;
+          break;
+        }
+        // Thread (w, lane) writes 16 columns of one row: row slot_row / 4,
+        // columns 16 * (slot_row % 4) ...
+        const int row = slot_row >> 2, q4 = slot_row & 3;
+        if (row < U.rows) {
+          float2 ml[4];
+          float mx = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            ml[w] = q_ml[w * 32 + row];
+            if (ml[w].y > 0.f) mx = fmaxf(mx, ml[w].x);
+          }
+          float o[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) o[e] = 0.f;
+          float l = 0.f;
+          if (mx != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              if (ml[w].y > 0.f) {
+                const float wgt = ex2_approx(ml[w].x - mx);
+                l += ml[w].y * wgt;
+                const float4* src = reinterpret_cast<const float4*>(q_o + (w * 32 + row) * DH);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                  const float4 t4 = src[(q4 * 4 + v) ^ (row & 15)];
+                  o[4 * v] += t4.x * wgt;
+                  o[4 * v + 1] += t4.y * wgt;
+                  o[4 * v + 2] += t4.z * wgt;
+                  o[4 * v + 3] += t4.w * wgt;
+                }
+              }
+            }
+            if constexpr (EXT) {
+              if (p.sinks != nullptr) l += ex2_approx(__ldg(p.sinks + U.h) * kLog2e - mx);
+            }
+          }
+          const float inv = l > 0.f ? 1.f / l : 0.f;
+          uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<int64_t>(U.b) * p.t_q + U.q0 + row) * p.out_stride +
+                                                U.h * DH + 16 * q4);
+#pragma unroll
+          for (int v = 0; v < 2; ++v) {
+            uint4 w4;
+            w4.x = pack_half2(o[8 * v + 0] * inv, o[8 * v + 1] * inv);
+            w4.y = pack_half2(o[8 * v + 2] * inv, o[8 * v + 3] * inv);
+            w4.z = pack_half2(o[8 * v + 4] * inv, o[8 * v + 5] * inv);
+            w4.w = pack_half2(o[8 * v + 6] * inv, o[8 * v + 7] * inv);
+            dst[v] = w4;
+          }
+        }
+        continue;
+      }
       // A sink adds 2^(sink*log2e - m) to the normaliser (split partials get it
       // in the combine step). No visible key: m = -inf, so the output is 0.
       float l_fin = l_run;

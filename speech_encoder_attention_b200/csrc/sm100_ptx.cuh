@@ -203,6 +203,14 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// Pulls a tile of a 3-D tensor map into L2 (no shared memory, no barrier).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int32_t c0, int32_t c1, int32_t c2) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                             int32_t c0, int32_t c1) {
   asm volatile(
@@ -426,96 +434,6 @@ __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// 16-lane shapes. A warp reads or writes 16 consecutive lanes of its lane
-// quadrant (the lane field of taddr); each repetition covers the next columns.
-//   16x256b (8 columns of 32 bits per repetition): thread t holds, for lanes
-//     base + t/4 and base + t/4 + 8, columns 2(t%4) and 2(t%4)+1, in the
-//     register order (t/4, c), (t/4, c+1), (t/4+8, c), (t/4+8, c+1).
-//   16x128b (4 columns per repetition): thread t holds column t%4 of lanes
-//     base + t/4 and base + t/4 + 8, in that order.
-// So a row's values sit in four consecutive threads (a quad), and a row
-// reduction is two xor-shuffles.
-
-#define SEA_R8(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), "=r"(r[i + 4]), \
-                  "=r"(r[i + 5]), "=r"(r[i + 6]), "=r"(r[i + 7])
-#define SEA_RW8(i) "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]), "+r"(r[i + 4]), \
-                   "+r"(r[i + 5]), "+r"(r[i + 6]), "+r"(r[i + 7])
-#define SEA_IN8(i) "r"(r[i]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3]), "r"(r[i + 4]), \
-                   "r"(r[i + 5]), "r"(r[i + 6]), "r"(r[i + 7])
-
-// 16 lanes x 128 columns, without waiting: the registers are only valid after
-// tmem_wait_ld64 on the same array.
-__device__ __forceinline__ void tmem_ld16x256b_x16(uint32_t taddr, uint32_t (&r)[64]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.16x256b.x16.b32"
-      " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15,"
-      " %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31,"
-      " %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47,"
-      " %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];"
-      : SEA_R8(0), SEA_R8(8), SEA_R8(16), SEA_R8(24), SEA_R8(32), SEA_R8(40), SEA_R8(48), SEA_R8(56)
-      : "r"(taddr)
-      : "memory");
-}
-
-// Waits for this thread's outstanding tensor-memory loads; naming the
-// destination registers as read-write operands keeps the compiler from
-// touching them before the wait.
-__device__ __forceinline__ void tmem_wait_ld64(uint32_t (&r)[64]) {
-  asm volatile("tcgen05.wait::ld.sync.aligned;"
-               : SEA_RW8(0), SEA_RW8(8), SEA_RW8(16), SEA_RW8(24), SEA_RW8(32), SEA_RW8(40), SEA_RW8(48),
-                 SEA_RW8(56)
-               :
-               : "memory");
-}
-
-// 16 lanes x 64 columns, waiting for the load.
-__device__ __forceinline__ void tmem_ld16x256b_x8(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.16x256b.x8.b32"
-      " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15,"
-      " %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : SEA_R8(0), SEA_R8(8), SEA_R8(16), SEA_R8(24)
-      : "r"(taddr)
-      : "memory");
-}
-
-// 16 lanes x 64 columns, waiting until the store is performed.
-__device__ __forceinline__ void tmem_st16x256b_x8(uint32_t taddr, const uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.16x256b.x8.b32 [%0],"
-      " {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16,"
-      " %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};\n\t"
-      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
-      SEA_IN8(0), SEA_IN8(8), SEA_IN8(16), SEA_IN8(24)
-      : "memory");
-}
-
-// 16 lanes x 16 columns (four 16x128b repetitions), without waiting.
-__device__ __forceinline__ void tmem_st16x128b_x4(uint32_t taddr, const uint32_t (&r)[8]) {
-  asm volatile("tcgen05.st.sync.aligned.16x128b.x4.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
-               SEA_IN8(0)
-               : "memory");
-}
-
-// 32 lanes x 64 columns (thread = lane), waiting for the load.
-__device__ __forceinline__ void tmem_ld32x32b_x64(uint32_t taddr, uint32_t (&r)[64]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x64.b32"
-      " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15,"
-      " %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31,"
-      " %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47,"
-      " %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : SEA_R8(0), SEA_R8(8), SEA_R8(16), SEA_R8(24), SEA_R8(32), SEA_R8(40), SEA_R8(48), SEA_R8(56)
-      : "r"(taddr)
-      : "memory");
-}
-
-#undef SEA_R8
-#undef SEA_RW8
-#undef SEA_IN8
-
 // ---------------------------------------------------------------------------
 // descriptors
 // ---------------------------------------------------------------------------
@@ -579,40 +497,10 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   return d;
 }
 
-__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
-}
-
-// 2^x for a pair of arguments on the FMA and integer pipes (no MUFU): the
-// Cody-Waite split x = n + f with n = round(x) (the 1.5 * 2^23 shifter) and
-// f in [-1/2, 1/2], a cubic for 2^f (coefficients from a minimax fit of the
-// relative error by Remez exchange, fit_exp2_poly.py; max relative error
-// 7.5e-5), and 2^n applied by adding n to the exponent field. Arguments are
-// clamped to >= -125 so the exponent never underflows: the result is then at
-// most 2^-125 where the exact value is smaller, which is zero after the fp16
-// rounding of P and negligible in the fp32 row sum.
-__device__ __forceinline__ void exp2_poly_x2(float x0, float x1, float& p0, float& p1) {
-  const uint64_t x = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
-  const uint64_t shifter = f2_pack(12582912.f, 12582912.f);
-  const uint64_t t = f2_add(x, shifter);        // n in the low mantissa bits
-  const uint64_t f = f2_sub(x, f2_sub(t, shifter));
-  uint64_t q = f2_fma(f2_pack(0.0551716685295105f, 0.0551716685295105f), f,
-                      f2_pack(0.2426111251115799f, 0.2426111251115799f));
-  q = f2_fma(q, f, f2_pack(0.6932609677314758f, 0.6932609677314758f));
-  q = f2_fma(q, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));
-  float q0, q1, t0, t1;
-  f2_unpack(q, q0, q1);
-  f2_unpack(t, t0, t1);
-  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
-  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {

@@ -248,6 +248,19 @@ def test_plan_long_splits_use_the_workspace(lib):
     assert (p["kv_splits"], p["cluster_merge"], p["workspace_bytes"]) == (6, 1, 0)
 
 
+def test_plan_narrow_tiles_for_decode_sized_blocks(lib):
+    # the drafter: 5 beams x 16 queries, 20 heads -> 100 one-tile units, no split
+    p = attn.debug_plan(5, 16, 448, 20, num_sms=148)
+    assert (p["kv_splits"], p["units"], p["narrow"]) == (1, 100, 1)
+    assert attn.debug_plan(5, 32, 448, 20, num_sms=148)["narrow"] == 1      # up to 32 rows
+    assert attn.debug_plan(5, 33, 448, 20, num_sms=148)["narrow"] == 0      # more rows: the 128-row layout
+    assert attn.debug_plan(5, 16, 448, 20, attn.MASK_BAND, num_sms=148)["narrow"] == 1
+    assert attn.debug_plan(8, 16, 448, 20, num_sms=148)["narrow"] == 0      # 160 units: more than one per SM
+    p = attn.debug_plan(1, 16, 448, 20, num_sms=148)                         # 20 units: the key split instead
+    assert p["kv_splits"] > 1 and p["narrow"] == 0
+    assert attn.debug_plan(5, 16, 448, 20, attn.MASK_SLOTMASK, num_sms=148)["narrow"] == 0
+
+
 def test_plan_does_not_split_when_units_fill_the_gpu(lib):
     p = attn.debug_plan(1, 80, 1500, 80, num_sms=148)  # 80 units: more than half of 148
     assert p["kv_splits"] == 1 and p["workspace_bytes"] == 0

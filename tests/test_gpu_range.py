@@ -97,6 +97,43 @@ def test_causal_split_and_unsplit_agree_with_oracle(split):
 
 
 # ---------------------------------------------------------------------------
+# narrow query tiles (at most 32 rows: the rows in every lane quadrant, each
+# softmax warp a quarter of the key columns, four partials merged per row)
+# ---------------------------------------------------------------------------
+
+NARROW_CASES = [  # (t_q, t_kv, batch, heads, options)
+    (1, 1, 3, 2, {}), (1, 700, 3, 2, {}), (7, 129, 5, 3, {}), (16, 448, 5, 4, {}), (31, 1000, 2, 2, {}),
+    (32, 256, 4, 2, {}), (16, 448, 5, 4, {"causal": True}), (20, 10, 3, 2, {"causal": True}),
+    (32, 100, 2, 2, {"causal": True}), (16, 300, 4, 2, {"mask_kind": attn.MASK_BAND, "window": 50}),
+    (16, 448, 5, 2, {"sinks": [0.5, -1.0]}), (16, 448, 5, 2, {"sinks": [2.0, 0.0], "causal": True}),
+    (24, 500, 4, 2, {"q_lens": [24, 9, 0, 17], "kv_lens": [500, 33, 200, 0]}),
+]
+
+
+@pytest.mark.parametrize("case", range(len(NARROW_CASES)))
+def test_narrow_query_tiles(case):
+    t_q, t_kv, batch, heads, opts = NARROW_CASES[case]
+    # unsplit (the narrow layout needs one unit per CTA and no key split)
+    assert batch * heads <= 148 and t_q <= 32
+    rng = np.random.default_rng(900 + case)
+    q, k, v = rand_qkv(rng, batch, t_q, t_kv, heads)
+    got, _ = check(q, k, v, batch, t_q, t_kv, heads, f"narrow {t_q}x{t_kv} {opts}", split=False, **opts)
+    if opts.get("q_lens") is not None:
+        for b, n in enumerate(opts["q_lens"]):
+            np.testing.assert_array_equal(got[b * t_q + n:(b + 1) * t_q], 0.0)
+
+
+def test_narrow_and_wide_layouts_agree():
+    """33 rows take the 128-row layout, 32 the narrow one: the first 32 rows
+    of a 33-row block (FULL, no split) match the 32-row block within rounding."""
+    rng = np.random.default_rng(77)
+    q, k, v = rand_qkv(rng, 1, 33, 600, 2)
+    wide = run(q, k, v, 1, 33, 600, 2, split=False)
+    narrow = run(q[:32], k, v, 1, 32, 600, 2, split=False)
+    assert_parity(narrow, wide[:32], rel_tol=1e-3, abs_tol=2e-3, what="narrow vs wide")
+
+
+# ---------------------------------------------------------------------------
 # band (sliding window)
 # ---------------------------------------------------------------------------
 
