@@ -581,9 +581,12 @@ __global__ void __launch_bounds__(CfgT<STAGES>::THREADS, STAGES == 2 ? 2 : 1)
           for (int e = 0; e < 128; ++e)
             if (!((wbits[e >> 5] >> (e & 31)) & 1u) || e >= lim) s[e] = -INFINITY;
         } else {
+          // Keys outside the row's range [lo_i, hi_i). Rows past the tile's
+          // rows are never stored and need no mask (their scores are finite:
+          // zero-filled or real rows).
           const int a = lo_i - kv0;
           const int bnd = hi_i - kv0;
-          if (a > 0 || bnd < NC) {
+          if (row_ok && (a > 0 || bnd < NC)) {
 #pragma unroll
             for (int e = 0; e < NC; ++e)
               if (e < a || e >= bnd) s[e] = -INFINITY;
