@@ -587,9 +587,17 @@ __global__ void __launch_bounds__(CfgT<STAGES>::THREADS, STAGES == 2 ? 2 : 1)
           const int a = lo_i - kv0;
           const int bnd = hi_i - kv0;
           if (row_ok && (a > 0 || bnd < NC)) {
+            if (a <= 0 && bnd >= NC / 2) {
+              // Only the end of the range falls in the tile's upper half
+              // (the last key tile of a full-range row).
 #pragma unroll
-            for (int e = 0; e < NC; ++e)
-              if (e < a || e >= bnd) s[e] = -INFINITY;
+              for (int e = NC / 2; e < NC; ++e)
+                if (e >= bnd) s[e] = -INFINITY;
+            } else {
+#pragma unroll
+              for (int e = 0; e < NC; ++e)
+                if (e < a || e >= bnd) s[e] = -INFINITY;
+            }
           }
         }
         // The tile's row max: four independent chains of 3-input max.
