@@ -255,36 +255,46 @@ class EncoderStep:
         self.lens = None if lens is None else dev(lens)
         self.host_x = torch.from_numpy(inp.x).pin_memory()
         self.host_out = torch.empty(rows, d, dtype=torch.float16).pin_memory()
+        self.x_sets = [self.x, self.x.clone()]
+        self.out_sets = [self.out, torch.empty_like(self.out)]
+        self.host_out_sets = [self.host_out, torch.empty(rows, d, dtype=torch.float16).pin_memory()]
         self.kernels = ["qkv_gemm", "flash_attn"]
         # algorithmic work: the projection of the valid frames, attention over allowed pairs
         self.flops = {"qkv_gemm": qkv_flops(encoder_valid_rows(spec), d),
                       "flash_attn": attn_pair_flops(encoder_pairs(spec), spec.n_heads)}
         self.launches_per_step = 2
 
-    def run(self, events=None):
+    def run(self, events=None, x=None, out=None):
         # Direct launches: a CUDA graph of the two calls measured ~9 us slower
         # per step than these (programmatic launch of the attention grid
         # during the projection's last wave).
         a, d, s = self.attn, self.d, self.spec
         if events:
             events[0].record()
-        a.attn_qkv_pack(self.x, self.w, self.bq, self.bv, out=self.qkv)
+        a.attn_qkv_pack(self.x if x is None else x, self.w, self.bq, self.bv, out=self.qkv)
         if events:
             events[1].record()
         a.attn_forward(self.qkv[:, :d], self.qkv[:, d:2 * d], self.qkv[:, 2 * d:], s.batch, s.t, s.t, s.n_heads,
                        mask_kind=self.mask, chunk_len=s.chunk_len, window=s.band, q_lens=self.lens,
-                       kv_lens=self.lens, out=self.out, split=False)
+                       kv_lens=self.lens, out=self.out if out is None else out, split=False)
         if events:
             events[2].record()
 
-    def run_e2e(self, events=None):
-        if events:
-            events[0].record()
-        self.x.copy_(self.host_x, non_blocking=True)
-        self.run()
-        self.host_out.copy_(self.out, non_blocking=True)
-        if events:
-            events[-1].record()
+    # end to end: two sets of input / output buffers (the projection's output
+    # is an intermediate of the compute stream alone)
+    e2e_sets = 2
+
+    def e2e_in(self, b):
+        self.x_sets[b].copy_(self.host_x, non_blocking=True)
+
+    def e2e_compute(self, b):
+        self.run(x=self.x_sets[b], out=self.out_sets[b])
+
+    def e2e_out(self, b):
+        self.host_out_sets[b].copy_(self.out_sets[b], non_blocking=True)
+
+    def e2e_read_back_matches(self, b):
+        return bool((self.host_out_sets[b] == self.out_sets[b].cpu()).all())
 
     @property
     def h2d_bytes(self):
@@ -442,17 +452,25 @@ class VerifyStep:
     def run_split(self, events):
         self.graphs.run_split(events)
 
-    def run_e2e(self, events=None):
-        i = self.graphs.next_copy()
-        c = self.copies[i]
-        if events:
-            events[0].record()
-        c["q"].copy_(self.host_q, non_blocking=True)
-        self.graphs.run(copy=i)
-        self.host_out[:self.spec.t_q].copy_(c["o_self"], non_blocking=True)
-        self.host_out[self.spec.t_q:].copy_(c["o_cross"], non_blocking=True)
-        if events:
-            events[-1].record()
+    # end to end: every device copy is one buffer set
+    @property
+    def e2e_sets(self):
+        return self.graphs.n
+
+    def e2e_in(self, b):
+        self.copies[b]["q"].copy_(self.host_q, non_blocking=True)
+
+    def e2e_compute(self, b):
+        self.graphs.run(copy=b)
+
+    def e2e_out(self, b):
+        self.host_out[:self.spec.t_q].copy_(self.copies[b]["o_self"], non_blocking=True)
+        self.host_out[self.spec.t_q:].copy_(self.copies[b]["o_cross"], non_blocking=True)
+
+    def e2e_read_back_matches(self, b):
+        import torch
+        dev = torch.cat([self.copies[b]["o_self"], self.copies[b]["o_cross"]]).cpu()
+        return bool((self.host_out == dev).all())
 
     @property
     def h2d_bytes(self):
@@ -518,16 +536,21 @@ class DrafterStep:
     def run_split(self, events):
         self.graphs.run_split(events)
 
-    def run_e2e(self, events=None):
-        i = self.graphs.next_copy()
-        c = self.copies[i]
-        if events:
-            events[0].record()
-        c["q"].copy_(self.host_q, non_blocking=True)
-        self.graphs.run(copy=i)
-        self.host_out.copy_(c["out"], non_blocking=True)
-        if events:
-            events[-1].record()
+    @property
+    def e2e_sets(self):
+        return self.graphs.n
+
+    def e2e_in(self, b):
+        self.copies[b]["q"].copy_(self.host_q, non_blocking=True)
+
+    def e2e_compute(self, b):
+        self.graphs.run(copy=b)
+
+    def e2e_out(self, b):
+        self.host_out.copy_(self.copies[b]["out"], non_blocking=True)
+
+    def e2e_read_back_matches(self, b):
+        return bool((self.host_out == self.copies[b]["out"].cpu()).all())
 
     @property
     def h2d_bytes(self):
@@ -585,16 +608,21 @@ class Q8Step:
     def run_split(self, events):
         self.graphs.run_split(events)
 
-    def run_e2e(self, events=None):
-        i = self.graphs.next_copy()
-        c = self.copies[i]
-        if events:
-            events[0].record()
-        c["x"].copy_(self.host_x, non_blocking=True)
-        self.graphs.run(copy=i)
-        self.host_out.copy_(c["out"], non_blocking=True)
-        if events:
-            events[-1].record()
+    @property
+    def e2e_sets(self):
+        return self.graphs.n
+
+    def e2e_in(self, b):
+        self.copies[b]["x"].copy_(self.host_x, non_blocking=True)
+
+    def e2e_compute(self, b):
+        self.graphs.run(copy=b)
+
+    def e2e_out(self, b):
+        self.host_out.copy_(self.copies[b]["out"], non_blocking=True)
+
+    def e2e_read_back_matches(self, b):
+        return bool((self.host_out == self.copies[b]["out"].cpu()).all())
 
     @property
     def h2d_bytes(self):
@@ -875,6 +903,62 @@ def time_steps(step, flush, steps, warmup, clocks=None, barrier=None):
     return step_ms, per_kernel, latency_ms
 
 
+def time_e2e(step, steps, warmup, barrier=None):
+    """End-to-end steps through the same library calls with host buffers.
+    Step i copies its input from pinned host memory into buffer set i mod B
+    on a copy-in stream, runs its calls on the compute stream once that copy
+    has landed, and reads its result back into pinned host memory on a
+    copy-out stream once they are done. A set is written again only after
+    the step that used it B steps earlier has been computed (input) and read
+    back (output), so neighbouring steps' copies overlap the compute, as a
+    streaming pipeline runs them. Timed from before the first copy to after
+    the last read-back. Returns ms per step."""
+    import torch
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    nb = step.e2e_sets
+    ev = lambda: torch.cuda.Event()
+    in_done, comp_done, out_done = [ev() for _ in range(nb)], [ev() for _ in range(nb)], [ev() for _ in range(nb)]
+
+    def run(n):
+        s_in.wait_stream(comp)
+        for i in range(n):
+            b = i % nb
+            with torch.cuda.stream(s_in):
+                if i >= nb:
+                    s_in.wait_event(comp_done[b])  # the step that read this input set is done
+                step.e2e_in(b)
+                in_done[b].record(s_in)
+            comp.wait_event(in_done[b])
+            if i >= nb:
+                comp.wait_event(out_done[b])  # this output set has been read back
+            step.e2e_compute(b)
+            comp_done[b].record(comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(comp_done[b])
+                step.e2e_out(b)
+                out_done[b].record(s_out)
+        comp.wait_stream(s_out)
+        comp.wait_stream(s_in)
+
+    run(max(1, warmup))
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if barrier is not None:
+        barrier()
+    torch.cuda.synchronize()
+    start.record(comp)
+    run(steps)
+    end.record(comp)
+    torch.cuda.synchronize()
+    if barrier is not None:
+        barrier()
+    # the last read-back holds the last step's result
+    if not step.e2e_read_back_matches((steps - 1) % nb):
+        raise RuntimeError("end-to-end read-back differs from the device result: stream ordering is broken")
+    return start.elapsed_time(end) / steps
+
+
 def time_secondary(name, device, steps, warmup, ws):
     """The bandwidth-bound verify step (token-tree SLOTMASK + cross-attention),
     timed like a `--workload verify` run (data cold in HBM, CUDA events on the
@@ -929,19 +1013,9 @@ def run_gpu(args):
     # end to end through the same calls, host buffers, copies inside the timed region
     e2e_ms = None
     if not args.skip_e2e:
-        for _ in range(max(1, args.warmup // 2)):
-            step.run_e2e()
-        torch.cuda.synchronize()
         n_e2e = max(1, min(args.steps, args.e2e_steps))
-        eev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n_e2e)]
-        barrier()
-        torch.cuda.synchronize()
-        for i in range(n_e2e):
-            step.run_e2e(eev[i])
-        torch.cuda.synchronize()
-        barrier()
+        e2e_local = time_e2e(step, n_e2e, max(2, args.warmup // 2), barrier)
         check_device_errors(step, "end-to-end steps")
-        e2e_local = sum(a.elapsed_time(b) for a, b in eev) / n_e2e
         e2e_ms = reduce_step_time(e2e_local, device)
 
     # the bandwidth-bound decoder step, reported beside the encoder headline
@@ -1014,7 +1088,9 @@ def run_gpu(args):
         "e2e": None if e2e_ms is None else {
             "value": whole_job_rate(flops, ws, e2e_ms) / 1e12, "unit": unit,
             "h2d_bytes_per_step": step.h2d_bytes, "d2h_bytes_per_step": step.d2h_bytes,
-            "ms_per_step": e2e_ms},
+            "ms_per_step": e2e_ms,
+            "timing": ("steps pipelined over a copy-in, a compute and a copy-out stream with "
+                       f"{step.e2e_sets} buffer sets; pinned host memory; first copy to last read-back")},
         "secondary": secondary,
         "gpu_launches": step.launches_per_step * args.steps,
         "timing": STEP_TIMING_COLD if getattr(step, "cold", False) else STEP_TIMING_FLUSHED,
