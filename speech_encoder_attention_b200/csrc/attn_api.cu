@@ -208,6 +208,17 @@ constexpr int kMaxClusterSplits = 8;
 
 int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
 
+// Multiplier and shift for sea::fa::div_c (division by a launch constant).
+sea::fa::DivC make_divc(int d) {
+  sea::fa::DivC f{0u, 0u, d};
+  if (d <= 1) return f;
+  int l = 0;
+  while ((int64_t(1) << l) < d) ++l;  // ceil(log2 d)
+  f.m = static_cast<uint32_t>(((uint64_t(1) << (31 + l)) + static_cast<uint64_t>(d) - 1) / static_cast<uint64_t>(d));
+  f.s = static_cast<uint32_t>(l - 1);
+  return f;
+}
+
 // Launch plan shared by attn_forward and attn_workspace_size.
 FaPlan plan_forward(int batch, int t_q, int t_kv, int n_heads, int mask_kind, int chunk_len, int num_sms) {
   FaPlan pl{};
@@ -419,6 +430,11 @@ attn_status launch_attention(attn_mat q, attn_mat k, attn_mat v, int32_t batch, 
   p.q_tiles = pl.q_tiles;
   p.kv_splits = pl.kv_splits;
   p.kv_tiles_per_split = pl.kv_tiles_per_split;
+  p.dv_splits = make_divc(p.kv_splits);
+  p.dv_q_tiles = make_divc(p.q_tiles);
+  p.dv_heads = make_divc(p.n_heads);
+  p.dv_tiles_per_seg = make_divc(p.tiles_per_seg);
+  p.dv_chunk = make_divc(p.chunk_len);
   p.out = static_cast<__half*>(out.ptr);
   p.out_stride = out.row_stride;
   float* ws = static_cast<float*>(workspace);

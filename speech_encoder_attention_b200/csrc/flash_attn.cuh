@@ -52,6 +52,21 @@ constexpr int MAX_FLAG_WORDS = 16;        // SLOTMASK: up to 512 key tiles (6553
 
 enum MaskKind : int { kFull = 0, kChunk = 1, kSlotmask = 2, kBand = 3 };
 
+// Division by a launch constant d >= 1 without the integer-divide sequence
+// (its reciprocal runs on MUFU, which the softmax keeps saturated): for
+// 0 <= n < 2^31, n / d = umulhi(n, m) >> s with l = ceil(log2 d),
+// m = ceil(2^(31 + l) / d) and s = l - 1 (division by invariant integers
+// using multiplication, Granlund and Montgomery); d = 1 is m = 0. The host
+// fills m and s.
+struct DivC {
+  uint32_t m, s;
+  int d;
+};
+
+__device__ __forceinline__ int div_c(int n, const DivC& f) {
+  return f.m ? static_cast<int>(__umulhi(static_cast<uint32_t>(n), f.m) >> f.s) : n;
+}
+
 struct Params {
   int batch, t_q, t_kv, n_heads;
   float scale_log2;  // scale * log2(e)
@@ -73,6 +88,8 @@ struct Params {
   int kv_splits, kv_tiles_per_split;
   // work units: batch * n_heads * q_tiles * kv_splits (split fastest)
   int units;
+  // the divisions by kv_splits, q_tiles, n_heads, tiles_per_seg, chunk_len
+  DivC dv_splits, dv_q_tiles, dv_heads, dv_tiles_per_seg, dv_chunk;
   // outputs
   __half* out;
   int64_t out_stride;
@@ -130,7 +147,7 @@ struct TileGeom {
 __device__ __forceinline__ TileGeom q_tile_geom(const Params& p, int qt) {
   TileGeom g{p.t_q, 0};
   if (qt >= p.q_tiles) return g;
-  const int seg = qt / p.tiles_per_seg;
+  const int seg = div_c(qt, p.dv_tiles_per_seg);
   const int w = qt - seg * p.tiles_per_seg;
   const int seg0 = seg * p.seg_len;
   const int q0 = seg0 + w * BQ;
@@ -167,7 +184,7 @@ __device__ __forceinline__ void row_keys(const Params& p, const SeqLen& L, int i
   hi = L.kv;
   if constexpr (!EXT) {
     if (p.mask_kind == kChunk) {
-      lo = (i / p.chunk_len) * p.chunk_len;
+      lo = div_c(i, p.dv_chunk) * p.chunk_len;
       hi = min(hi, lo + p.chunk_len);
     }
     return;
@@ -182,7 +199,7 @@ __device__ __forceinline__ void row_keys(const Params& p, const SeqLen& L, int i
       hi = 0;
       return;
     }
-    lo = (pos / p.chunk_len) * p.chunk_len;
+    lo = div_c(pos, p.dv_chunk) * p.chunk_len;
     hi = min(hi, lo + p.chunk_len);
   } else if (p.mask_kind == kBand) {
     lo = max(0, pos - p.window + 1);
@@ -202,12 +219,12 @@ struct Unit {
 template <bool EXT>
 __device__ __forceinline__ Unit decode_unit(const Params& p, int u) {
   Unit U;
-  U.split = u % p.kv_splits;
-  int r = u / p.kv_splits;
-  const int qt = r % p.q_tiles;
-  r /= p.q_tiles;
-  U.h = r % p.n_heads;
-  U.b = r / p.n_heads;
+  int r = div_c(u, p.dv_splits);
+  U.split = u - r * p.kv_splits;
+  const int r2 = div_c(r, p.dv_q_tiles);
+  const int qt = r - r2 * p.q_tiles;
+  U.b = div_c(r2, p.dv_heads);
+  U.h = r2 - U.b * p.n_heads;
   const TileGeom g = q_tile_geom(p, qt);
   U.q0 = g.q0;
   U.rows = g.rows;

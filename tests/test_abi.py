@@ -5,6 +5,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 from speech_encoder_attention_b200 import attn
@@ -292,3 +293,25 @@ def test_static_scratch_rejects_invalid_arguments_before_any_cuda_call(lib, kw):
     at the device: here, with no usable device, an invalid call must still say
     ATTN_ERR_INVALID (a device query would have failed with another status)."""
     assert call_static_scratch(lib, **kw) == attn.ATTN_ERR_INVALID
+
+
+def test_division_by_launch_constants():
+    """The attention kernels divide by launch constants (key splits, query
+    tiles, heads, chunk length) as umulhi(n, m) >> s with l = ceil(log2 d),
+    m = ceil(2^(31 + l) / d), s = l - 1 (the host computes m and s): exact for
+    every 0 <= n < 2^31, checked here densely at both ends of that range."""
+    def magic(d):
+        if d <= 1:
+            return 0, 0
+        l = (d - 1).bit_length()
+        return ((1 << (31 + l)) + d - 1) // d, l - 1
+
+    rng = np.random.default_rng(3)
+    divisors = list(range(1, 2049)) + [2 ** k + e for k in range(11, 31) for e in (-1, 0, 1)] + [2 ** 31 - 1]
+    for d in divisors:
+        m, s = magic(d)
+        assert m < 2 ** 32
+        n = np.concatenate([np.arange(0, 600), np.arange(2 ** 31 - 600, 2 ** 31),
+                            rng.integers(0, 2 ** 31, 200)]).astype(object)
+        q = n if m == 0 else ((n * m) >> 32) >> s
+        assert all(q == n // d), d
