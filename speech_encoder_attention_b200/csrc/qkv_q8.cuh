@@ -13,9 +13,12 @@
 // the SMs even for a single row tile.
 //
 // Design (192 threads per CTA):
-//   warp 0      TMA producer: per K step of 256 weights, x as four 64-column
-//               slices (128-byte swizzle) and the 32 weight rows' 8 blocks
-//               (272 raw bytes each) into a 2-stage ring.
+//   warp 0      TMA producer: the 32 weight rows' 8 blocks per K step of 256
+//               weights (272 raw bytes each) into a 6-stage ring whose first
+//               loads all start at once (a CTA reads each weight byte once,
+//               from HBM, so their latency is paid once rather than per K
+//               step), and per K step x as four 64-column slices (128-byte
+//               swizzle) into a 2-stage ring.
 //   warp 1      tcgen05.mma issuer (one thread): 128x32x16 f16 MMAs into 32
 //               fp32 tensor-memory columns.
 //   warps 2..5  dequantize each stage's raw blocks into an fp16 operand tile in
@@ -35,21 +38,23 @@ constexpr int BKQ = 256;                  // weights per K step (8 Q8_0 blocks)
 constexpr int QBLOCK = 32;                // weights per Q8_0 block
 constexpr int QBLOCK_BYTES = 34;          // fp16 scale + 32 int8
 constexpr int RAW_ROW_BYTES = (BKQ / QBLOCK) * QBLOCK_BYTES;  // 272
-constexpr int STAGES = 2;
+constexpr int STAGES = 2;                 // x and dequantized-operand ring
+constexpr int WSTAGES = 6;                // raw weight-block ring
 constexpr int A_BYTES = BM * BKQ * 2;     // 64 KB: four 128x64 fp16 slices
 constexpr int A_SLICE = BM * 64 * 2;      // 16 KB
 constexpr int RAW_BYTES = BN * RAW_ROW_BYTES;  // 8704
 constexpr int RAW_PAD = 9216;
 constexpr int B_BYTES = BN * BKQ * 2;     // 16 KB: four 32x64 fp16 slices
 constexpr int B_SLICE = BN * 64 * 2;      // 4 KB
-constexpr int STAGE_BYTES = A_BYTES + RAW_PAD + B_BYTES;
 constexpr int THREADS = 192;
 constexpr int TMEM_COLS = 32;
 
-constexpr int OFF_STAGES = 0;
-constexpr int OFF_BARS = OFF_STAGES + STAGES * STAGE_BYTES;
-// a_full[S], raw_full[S], b_ready[S], empty[S], acc_full, drain
-constexpr int NUM_BARS = 4 * STAGES + 2;
+constexpr int OFF_A = 0;                              // [STAGES] x tiles
+constexpr int OFF_B = OFF_A + STAGES * A_BYTES;       // [STAGES] dequantized W operands
+constexpr int OFF_RAW = OFF_B + STAGES * B_BYTES;     // [WSTAGES] raw weight blocks
+constexpr int OFF_BARS = OFF_RAW + WSTAGES * RAW_PAD;
+// a_full[S], b_ready[S], ab_empty[S], raw_full[W], raw_empty[W], acc_full, drain
+constexpr int NUM_BARS = 3 * STAGES + 2 * WSTAGES + 2;
 constexpr int OFF_MISC = OFF_BARS + 8 * NUM_BARS;
 constexpr int SMEM_BYTES = 1024 + OFF_MISC + 16;
 
@@ -71,14 +76,15 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + OFF_BARS;
   auto a_full = [&](int s) { return bar0 + 8u * s; };
-  auto raw_full = [&](int s) { return bar0 + 8u * (STAGES + s); };
-  auto b_ready = [&](int s) { return bar0 + 8u * (2 * STAGES + s); };
-  auto empty_bar = [&](int s) { return bar0 + 8u * (3 * STAGES + s); };
-  const uint32_t acc_full = bar0 + 8u * (4 * STAGES);
+  auto b_ready = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto ab_empty = [&](int s) { return bar0 + 8u * (2 * STAGES + s); };  // MMA done with x and B of stage s
+  auto raw_full = [&](int w) { return bar0 + 8u * (3 * STAGES + w); };
+  auto raw_empty = [&](int w) { return bar0 + 8u * (3 * STAGES + WSTAGES + w); };
+  const uint32_t acc_full = bar0 + 8u * (3 * STAGES + 2 * WSTAGES);
   const uint32_t drain_bar = acc_full + 8u;
-  auto stage_a = [&](int s) { return sbase + OFF_STAGES + s * STAGE_BYTES; };
-  auto stage_raw = [&](int s) { return stage_a(s) + A_BYTES; };
-  auto stage_b = [&](int s) { return stage_a(s) + A_BYTES + RAW_PAD; };
+  auto stage_a = [&](int s) { return sbase + OFF_A + s * A_BYTES; };
+  auto stage_b = [&](int s) { return sbase + OFF_B + s * B_BYTES; };
+  auto stage_raw = [&](int w) { return sbase + OFF_RAW + w * RAW_PAD; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC + 4);
 
@@ -91,9 +97,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(a_full(s), 1);
-      mbar_init(raw_full(s), 1);
       mbar_init(b_ready(s), 4);
-      mbar_init(empty_bar(s), 1);
+      mbar_init(ab_empty(s), 1);
+    }
+    for (int w = 0; w < WSTAGES; ++w) {
+      mbar_init(raw_full(w), 1);
+      mbar_init(raw_empty(w), 4);
     }
     mbar_init(acc_full, 1);
     mbar_init(drain_bar, 1);
@@ -118,23 +127,35 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer ----------------
-      int issued = 0;
-      for (int kb = 0; kb < ksteps; ++kb) {
+      // Raw blocks of K step kb into slot kb % WSTAGES once the dequantization
+      // of step kb - WSTAGES has read it (the raw map counts 2-byte units:
+      // 136 per 8 blocks).
+      int issued_w = 0, issued = 0;
+      auto load_w = [&](int kb) -> bool {
+        const int w = kb % WSTAGES;
+        if (kb >= WSTAGES && !mbar_wait(raw_empty(w), ((kb / WSTAGES) - 1) & 1, wc)) return false;
+        mbar_arrive_expect_tx(raw_full(w), RAW_BYTES);
+        tma_load_2d(stage_raw(w), &tm_w, raw_full(w), kb * (RAW_ROW_BYTES / 2), n0);
+        ++issued_w;
+        return true;
+      };
+      bool ok = true;
+      for (int kb = 0; kb < min(ksteps, WSTAGES) && ok; ++kb) ok = load_w(kb);
+      for (int kb = 0; kb < ksteps && ok; ++kb) {
         const int s = kb % STAGES;
-        if (!mbar_wait(empty_bar(s), ((kb / STAGES) & 1) ^ 1u, wc)) break;
+        if (!mbar_wait(ab_empty(s), ((kb / STAGES) & 1) ^ 1u, wc)) break;
         mbar_arrive_expect_tx(a_full(s), A_BYTES);
 #pragma unroll
         for (int a = 0; a < BKQ / 64; ++a)
           tma_load_2d(stage_a(s) + a * A_SLICE, &tm_x, a_full(s), kb * BKQ + a * 64, m0);
-        // the raw map counts 2-byte units: 136 per 8 blocks
-        mbar_arrive_expect_tx(raw_full(s), RAW_BYTES);
-        tma_load_2d(stage_raw(s), &tm_w, raw_full(s), kb * (RAW_ROW_BYTES / 2), n0);
         ++issued;
+        if (kb + WSTAGES < ksteps) ok = load_w(kb + WSTAGES);
       }
-      for (int i = max(0, issued - STAGES); i < issued; ++i) {
+      // Let the last copies land before the CTA may exit.
+      for (int i = max(0, issued - STAGES); i < issued; ++i)
         mbar_wait_drain(a_full(i % STAGES), (i / STAGES) & 1, args.limit_ns);
-        mbar_wait_drain(raw_full(i % STAGES), (i / STAGES) & 1, args.limit_ns);
-      }
+      for (int i = max(0, issued_w - WSTAGES); i < issued_w; ++i)
+        mbar_wait_drain(raw_full(i % WSTAGES), (i / WSTAGES) & 1, args.limit_ns);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -156,7 +177,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint64_t bd = smem_desc_sw128(stage_b(s) + slice * B_SLICE + within * 32, 16, 1024);
           mma_f16_ss(tmem_base, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
         }
-        mma_commit(empty_bar(s));
+        mma_commit(ab_empty(s));
       }
       if (ok) mma_commit(acc_full);
       mma_commit(drain_bar);
@@ -169,21 +190,29 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int qq = t & 3;            // 64-weight quarter of the K step == operand slice
     bool ok = true;
     for (int kb = 0; kb < ksteps; ++kb) {
-      const int s = kb % STAGES;
-      if (!mbar_wait(raw_full(s), (kb / STAGES) & 1, wc)) {
+      const int s = kb % STAGES, w = kb % WSTAGES;
+      if (!mbar_wait(raw_full(w), (kb / WSTAGES) & 1, wc)) {
         ok = false;
         break;
       }
       // this thread's two blocks: 34-byte records, so 2-byte loads (plain C++
       // loads, ordered after the barrier wait, which the compiler may batch)
       const uint16_t* raw16 = reinterpret_cast<const uint16_t*>(
-          smem + (stage_raw(s) - sbase) + r * RAW_ROW_BYTES + 2 * qq * QBLOCK_BYTES);
+          smem + (stage_raw(w) - sbase) + r * RAW_ROW_BYTES + 2 * qq * QBLOCK_BYTES);
       const uint32_t dst_row = stage_b(s) + qq * B_SLICE + r * 128;
       uint16_t words[2][17];
 #pragma unroll
       for (int bb = 0; bb < 2; ++bb)
 #pragma unroll
         for (int i = 0; i < 17; ++i) words[bb][i] = raw16[bb * (QBLOCK_BYTES / 2) + i];
+      // the raw slot may be refilled once every warp has read it; the operand
+      // stage once the MMAs of step kb - STAGES are done
+      __syncwarp();
+      if (lane == 0) mbar_arrive(raw_empty(w));
+      if (kb >= STAGES && !mbar_wait(ab_empty(s), ((kb / STAGES) - 1) & 1, wc)) {
+        ok = false;
+        break;
+      }
 #pragma unroll
       for (int bb = 0; bb < 2; ++bb) {
         const float d = __half2float(__ushort_as_half(words[bb][0]));
