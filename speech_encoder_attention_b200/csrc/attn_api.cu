@@ -302,10 +302,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 
 // Row counts from which the projection runs on CTA pairs (256 x 256 tiles,
 // cta_group::2): large enough that the pair tiles fill the GPU.
-#ifndef SEA_PAIR_MIN_ROWS
-#define SEA_PAIR_MIN_ROWS 4096
-#endif
-constexpr int64_t kPairMinRows = SEA_PAIR_MIN_ROWS;
+constexpr int64_t kPairMinRows = 4096;
 constexpr int kPairTileN = 512;  // plan code for the pair kernel (tile 256 rows x 256 columns)
 
 // Projection tile width by estimated time: waves of 128x256 tiles against
