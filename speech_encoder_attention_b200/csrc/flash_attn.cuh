@@ -33,10 +33,14 @@
 // stores so the next unit's PV can start.
 // Tile skipping: CHUNK walks only the key range of the query tile's chunk(s);
 // SLOTMASK skips key tiles whose mask words are zero for every row of the CTA.
-// Split-KV: for short query blocks the key range is split over units; each
-// writes unnormalised O with its m and l to the workspace and a combine kernel
-// merges them. Every kernel here waits (griddepcontrol) after its prologue, so
-// programmatic launches overlap that prologue with the previous kernel.
+// Split-KV: for short query blocks the key range is split over units. Up to 8
+// splits of a query tile form a thread-block cluster and merge their
+// unnormalised partials through distributed shared memory; more write them to
+// the workspace and a combine kernel merges them. Query tiles of at most 32
+// rows take the narrow layout (their rows in every lane quadrant, each softmax
+// warp a quarter of the key columns, see NARROW below). Every kernel here
+// waits (griddepcontrol) after its prologue, so programmatic launches overlap
+// that prologue with the previous kernel.
 #pragma once
 
 #include "sm100_ptx.cuh"
