@@ -143,3 +143,41 @@ def test_kernel_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
     assert bench.kernel_source_hash() == h0
     src.write_text("int f(int x) {\n  return x + 2;\n}\n")
     assert bench.kernel_source_hash() != h0
+
+
+def test_clock_sampler_with_a_fake_nvml(monkeypatch):
+    """The bench's clock sampler, against a fake NVML module: it samples while
+    its region runs, reports the median clock and the union of the reasons
+    (idle dropped), and puts the interpreter's switch interval back."""
+    import sys
+    import threading
+    import time
+    import types
+
+    import bench
+    clocks = iter([1965, 1900, 1950] * 1000)
+    reasons = iter([0x4, 0x0, 0x1] * 1000)
+    lock = threading.Lock()
+
+    def clock(h, which):
+        with lock:
+            return next(clocks)
+
+    def event_reasons(h):
+        with lock:
+            return next(reasons)
+
+    fake = types.SimpleNamespace(
+        NVML_CLOCK_SM=0, nvmlInit=lambda: None, nvmlDeviceGetHandleByIndex=lambda i: object(),
+        nvmlDeviceGetMaxClockInfo=lambda h, w: 1965, nvmlDeviceGetClockInfo=clock,
+        nvmlDeviceGetCurrentClocksEventReasons=event_reasons)
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    before = sys.getswitchinterval()
+    sampler = bench.ClockSampler(0)
+    with sampler:
+        time.sleep(0.02)
+    assert sys.getswitchinterval() == before
+    rec = sampler.summary()
+    assert rec["samples"] >= 3 and rec["samples_under_load"] == rec["samples"]
+    assert rec["sm_max_mhz"] == 1965 and rec["sm_mhz"] in (1900, 1950, 1965)
+    assert rec["reasons"] == ["sw_power_cap"]
