@@ -138,22 +138,13 @@ REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_pow
 
 
 class ClockSampler:
-    """SM clock and clock-event reasons from NVML, polled on a thread while the
-    timed region runs. An SM-clock query takes ~1.5 ms on B200 (the reasons
-    ~0.25 ms), so a region of a few milliseconds holds only a few samples:
-    the thread polls without pause, the interpreter switches threads every
-    0.1 ms meanwhile (instead of every 5 ms) so the launching thread cannot
-    starve it, and __enter__ returns only once the first sample is in."""
-
-    def __init__(self, device_index: int, period_s: float = 0.0002):
+    def __init__(self, device_index: int, period_s: float = 0.001):
         self.period = period_s
         self.samples = []
         self.max_mhz = None
         self._stop = threading.Event()
-        self._first = threading.Event()
         self._thread = None
         self._nvml = None
-        self._switch = None
         try:
             import pynvml
             pynvml.nvmlInit()
@@ -168,46 +159,39 @@ class ClockSampler:
         while not self._stop.is_set():
             try:
                 sm = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                util = nv.nvmlDeviceGetUtilizationRates(self._h).gpu
                 try:
                     reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
                 except AttributeError:
                     reasons = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
-                self.samples.append((sm, reasons))
+                self.samples.append((sm, util, reasons))
             except Exception:
                 pass
-            self._first.set()
             self._stop.wait(self.period)
 
     def __enter__(self):
         if self._nvml is not None:
-            self._switch = sys.getswitchinterval()
-            sys.setswitchinterval(1e-4)
             self._thread = threading.Thread(target=self._run, daemon=True)
             self._thread.start()
-            self._first.wait(0.05)
         return self
 
     def __exit__(self, *exc):
         self._stop.set()
         if self._thread is not None:
             self._thread.join()
-        if self._switch is not None:
-            sys.setswitchinterval(self._switch)
 
     def summary(self):
-        """Median SM clock and the union of the reasons over the samples. The
-        sampler brackets only timed regions, which keep the GPU busy, so every
-        sample counts as taken under load."""
         if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
                     "note": "no NVML samples"}
-        mhz = sorted(s[0] for s in self.samples)
+        loaded = [s for s in self.samples if s[1] > 0] or self.samples
+        mhz = sorted(s[0] for s in loaded)
         bits = 0
-        for s in self.samples:
-            bits |= int(s[1])
+        for s in loaded:
+            bits |= int(s[2])
         reasons = [name for bit, name in REASON_BITS.items() if bits & bit and name != "gpu_idle"]
         return {"sm_mhz": mhz[len(mhz) // 2], "sm_max_mhz": self.max_mhz, "reasons": reasons,
-                "samples": len(self.samples), "samples_under_load": len(self.samples)}
+                "samples": len(self.samples), "samples_under_load": len(loaded)}
 
 
 # ---------------------------------------------------------------------------
